@@ -1,0 +1,140 @@
+"""Seeded synthetic inputs shared by the fp64 oracle and the GPU harness.
+
+This module holds the input recipe only: the workload shapes and a
+counter-based N(0,1) -> bf16 generator (``gen.c``). It contains none of the
+attention arithmetic, so both sides of every parity check can import it
+without sharing any code of the method.
+
+Tensors are returned as numpy ``uint16`` arrays of bf16 bit patterns in the
+``[B, H, T, D]`` layout (D innermost) that the pages' interface uses
+("注意力家族", section 最小语义实现: q is [B,H_q,T_q,D], k and v are
+[B,H_kv,T_k,D]). Tensor ids: Q=0, K=1, V=2.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gen.c")
+_LIB = os.path.join(_HERE, "libgqa_inputs.so")
+
+TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile gen.c into libgqa_inputs.so next to it (gcc, -O3, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O3", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.gqa_gen_normal_bf16.restype = ctypes.c_int
+        lib.gqa_gen_normal_bf16.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint64,
+                                            ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int]
+        lib.gqa_gen_key.restype = ctypes.c_uint64
+        lib.gqa_gen_key.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def normal_bf16(seed: int, tensor_id: int, shape, start: int = 0, threads: int | None = None,
+                out: np.ndarray | None = None) -> np.ndarray:
+    """Elements [start, start + prod(shape)) of stream (seed, tensor_id), as bf16 bits.
+
+    ``out`` may be a preallocated C-contiguous uint16 array (for example a
+    pinned host buffer viewed through numpy).
+    """
+    n = int(np.prod(shape, dtype=np.int64)) if len(shape) else 1
+    if out is None:
+        out = np.empty(shape, dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.flags["C_CONTIGUOUS"] and out.size == n
+    _load().gqa_gen_normal_bf16(int(seed), int(tensor_id), int(start), n,
+                                out.ctypes.data, int(threads or default_threads()))
+    return out
+
+
+def bf16_bits_to_f32(u16: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    return (np.asarray(u16, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bf16 (round-to-nearest-even), returning bit patterns.
+
+    Used to build hand-written fixtures (values that are exact in bf16)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+
+
+def scale_pow2_bf16(u16: np.ndarray, exponent: int) -> np.ndarray:
+    """Multiply bf16 values by 2**exponent. Exact for normal values that stay normal."""
+    f = bf16_bits_to_f32(u16) * np.float32(2.0 ** exponent)
+    out = f32_to_bf16_bits(f)
+    return out.reshape(np.shape(u16))
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape and recipe of one synthetic workload (seeded iid N(0,1) bf16)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Tq: int
+    Tk: int
+    D: int
+    q_pow2: int = 0      # Q multiplied by 2**q_pow2 after bf16 rounding
+    seed: int = 0
+
+    @property
+    def q_shape(self):
+        return (self.B, self.Hq, self.Tq, self.D)
+
+    @property
+    def kv_shape(self):
+        return (self.B, self.Hkv, self.Tk, self.D)
+
+    def make(self, threads: int | None = None, q_out=None, k_out=None, v_out=None):
+        """Generate (q, k, v) bf16 bit arrays for this workload."""
+        q = normal_bf16(self.seed, TENSOR_Q, self.q_shape, threads=threads, out=q_out)
+        if self.q_pow2:
+            q[...] = scale_pow2_bf16(q, self.q_pow2)
+        k = normal_bf16(self.seed, TENSOR_K, self.kv_shape, threads=threads, out=k_out)
+        v = normal_bf16(self.seed, TENSOR_V, self.kv_shape, threads=threads, out=v_out)
+        return q, k, v
+
+
+# The five workloads of the benchmark plan. Names state what each one is.
+TINY = Workload("tiny causal GQA B2 Hq4 Hkv2 T128 D64", 2, 4, 2, 128, 128, 64)
+GQA_PREFILL = Workload("GQA prefill B4 Hq32 Hkv8 T4096 D128", 4, 32, 8, 4096, 4096, 128)
+MQA_LONG = Workload("MQA long prefill B1 Hq32 Hkv1 T32768 D128", 1, 32, 1, 32768, 32768, 128)
+GQA_DECODE = Workload("GQA decode B64 Hq32 Hkv8 Tk32768 D128", 64, 32, 8, 1, 32768, 128)
+MHA_SUFFIX = Workload("MHA suffix B8 H16 Tq512 at 7680 over Tk8192 D128 Qx4", 8, 16, 16, 512, 8192, 128,
+                      q_pow2=2)
+
+WORKLOADS = {
+    "tiny": TINY,
+    "gqa_prefill": GQA_PREFILL,
+    "mqa_long": MQA_LONG,
+    "gqa_decode": GQA_DECODE,
+    "mha_suffix": MHA_SUFFIX,
+}

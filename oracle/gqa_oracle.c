@@ -1,0 +1,168 @@
+/*
+ * fp64 CPU oracle for causal grouped-query softmax attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the bench's
+ * CPU-baseline / reference arm may load this code. The product path (the
+ * CUDA library) never calls it and shares no code with it.
+ *
+ * What it computes, written out from the definition with no tiling, no
+ * online softmax and no reordering:
+ *
+ *   o_a = softmax( Q_a K_{g(a)}^T / sqrt(d_h) + M ) V_{g(a)}
+ *     -- "注意力家族" (wineandchord.com, attention variants), section 统一记号,
+ *        the o_a equation.
+ *   g(a) = floor(a / (H_q / H_kv)): consecutive query heads share a KV head
+ *     -- "Attention Architecture Evolution", section GQA, group(i) formula;
+ *        "注意力家族", section 最小语义实现 (repeat_interleave mapping).
+ *   M: causal mask with the suffix offset. Query row i sits at absolute
+ *      position (T_k - T_q) + i and sees keys j <= (T_k - T_q) + i; the key at
+ *      the query's own position is visible.
+ *     -- "注意力家族", section 最小语义实现 (query_pos / key_pos / future) and
+ *        section Mask 与增量位置; "A Visual Guide to Attention", section
+ *        "Which positions are visible?".
+ *   Scale 1/sqrt(D) with D the head dimension (the ABI allows an override).
+ *
+ * Precision: every input is a bf16 value, widened exactly to double; all
+ * arithmetic is double; nothing is rounded to a lower precision. Subtracting
+ * the row maximum before exp() does not change the mathematical result; it
+ * only keeps exp() finite in double. The natural-log LSE (m + ln l) is also
+ * returned, for the split-KV merge checks.
+ *
+ * Layout: q element (b,a,i,d) at b*q_sb + a*q_sh + i*D + d; k and v element
+ * (b,h,t,d) at b*k_sb + h*k_sh + t*D + d (likewise v_*). A row id is the flat
+ * index (b*H_q + a)*T_q + i. Rows are independent, so any subset can be
+ * computed exactly.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static inline double bf16_to_double(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int B, Hq, Hkv, Tq, Tk, D;
+    long long q_sb, q_sh, k_sb, k_sh, v_sb, v_sh;
+    double scale;
+    const long long* rows;
+    long long n_rows;
+    double* out;
+    double* lse;
+    long long next; /* shared work counter */
+} oracle_job;
+
+/* One output row: o[b,a,i,:] and its log-sum-exp. s holds T_k doubles. */
+static void oracle_row(const oracle_job* J, long long row, double* s, double* qd,
+                       double* o, double* lse_out) {
+    const int D = J->D;
+    const long long i = row % J->Tq;
+    const long long a = (row / J->Tq) % J->Hq;
+    const long long b = row / ((long long)J->Tq * J->Hq);
+    const long long group = J->Hq / J->Hkv;       /* H_q / H_kv query heads per KV head */
+    const long long g = a / group;                 /* g(a) */
+    const long long pos = (long long)(J->Tk - J->Tq) + i; /* absolute query position */
+
+    const uint16_t* qrow = J->q + b * J->q_sb + a * J->q_sh + i * D;
+    const uint16_t* kplane = J->k + b * J->k_sb + g * J->k_sh;
+    const uint16_t* vplane = J->v + b * J->v_sb + g * J->v_sh;
+
+    for (int d = 0; d < D; ++d) qd[d] = bf16_to_double(qrow[d]);
+
+    /* scores s_j = scale * <q_i, k_j> for visible keys j = 0..pos */
+    double m = -INFINITY;
+    for (long long j = 0; j <= pos; ++j) {
+        const uint16_t* krow = kplane + j * D;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += qd[d] * bf16_to_double(krow[d]);
+        s[j] = J->scale * acc;
+        if (s[j] > m) m = s[j];
+    }
+    /* softmax weights and normaliser */
+    double l = 0.0;
+    for (long long j = 0; j <= pos; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+    }
+    /* weighted sum of value rows */
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (long long j = 0; j <= pos; ++j) {
+        const uint16_t* vrow = vplane + j * D;
+        const double w = s[j];
+        for (int d = 0; d < D; ++d) o[d] += w * bf16_to_double(vrow[d]);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= l;
+    if (lse_out) *lse_out = m + log(l);
+}
+
+static void* oracle_worker(void* arg) {
+    oracle_job* J = (oracle_job*)arg;
+    double* s = (double*)malloc(sizeof(double) * (size_t)J->Tk);
+    double* qd = (double*)malloc(sizeof(double) * (size_t)J->D);
+    if (!s || !qd) {
+        free(s);
+        free(qd);
+        return (void*)1;
+    }
+    const long long chunk = 4;
+    for (;;) {
+        long long r0 = __atomic_fetch_add(&J->next, chunk, __ATOMIC_RELAXED);
+        if (r0 >= J->n_rows) break;
+        long long r1 = r0 + chunk < J->n_rows ? r0 + chunk : J->n_rows;
+        for (long long r = r0; r < r1; ++r)
+            oracle_row(J, J->rows[r], s, qd, J->out + r * J->D, J->lse ? J->lse + r : NULL);
+    }
+    free(s);
+    free(qd);
+    return NULL;
+}
+
+/*
+ * Compute n_rows output rows. rows[r] is a flat row id (b*H_q + a)*T_q + i.
+ * out is [n_rows][D] doubles; lse is [n_rows] doubles or NULL.
+ * scale <= 0 selects 1/sqrt(D). n_threads <= 0 selects one thread.
+ * Returns 0 on success, 1 on invalid arguments, 2 on allocation failure.
+ */
+int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                    int Hkv, int Tq, int Tk, int D, long long q_sb, long long q_sh,
+                    long long k_sb, long long k_sh, long long v_sb, long long v_sh, double scale,
+                    const long long* rows, long long n_rows, double* out, double* lse,
+                    int n_threads) {
+    if (!q || !k || !v || !out || (!rows && n_rows > 0)) return 1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || D <= 0) return 1;
+    if (Hq % Hkv != 0 || Tq > Tk) return 1; /* the pages' asserted preconditions */
+    const long long total = (long long)B * Hq * Tq;
+    for (long long r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return 1;
+
+    oracle_job J;
+    J.q = q; J.k = k; J.v = v;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Tq = Tq; J.Tk = Tk; J.D = D;
+    J.q_sb = q_sb; J.q_sh = q_sh; J.k_sb = k_sb; J.k_sh = k_sh; J.v_sb = v_sb; J.v_sh = v_sh;
+    J.scale = scale > 0.0 ? scale : 1.0 / sqrt((double)D);
+    J.rows = rows; J.n_rows = n_rows; J.out = out; J.lse = lse; J.next = 0;
+
+    if (n_threads <= 1) return oracle_worker(&J) ? 2 : 0;
+    if (n_threads > 512) n_threads = 512;
+    pthread_t th[512];
+    int started[512];
+    int rc = 0;
+    for (int t = 0; t < n_threads; ++t) started[t] = pthread_create(&th[t], NULL, oracle_worker, &J) == 0;
+    for (int t = 0; t < n_threads; ++t) {
+        if (!started[t]) continue;
+        void* ret = NULL;
+        pthread_join(th[t], &ret);
+        if (ret) rc = 2;
+    }
+    /* if no thread could start, do the work here */
+    int any = 0;
+    for (int t = 0; t < n_threads; ++t) any |= started[t];
+    if (!any) rc = oracle_worker(&J) ? 2 : 0;
+    return rc;
+}
