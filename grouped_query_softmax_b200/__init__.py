@@ -1,0 +1,194 @@
+"""Causal grouped-query softmax attention on B200 (sm_100a): Python binding of libgqa.
+
+Every step of the computation runs in the CUDA kernels of ``libgqa.so``; this
+module only marshals arguments across the C ABI declared in ``include/gqa.h``.
+The functions named ``gqa_*`` mirror the C entry points one to one (device
+pointers as integers, sizes, strides, a stream handle). ``attn_fwd`` and
+``attn_decode`` are conveniences for torch tensors: they check dtype, device and
+layout, allocate the outputs (and the decode workspace) with torch, and call the
+same entry points. PyTorch supplies device memory and streams only.
+
+There is no CPU fallback: importing this package fails loudly if the CUDA
+library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GqaError", "gqa_attn_fwd", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
+    "gqa_attn_decode_num_splits", "gqa_status_string", "gqa_get_device_error",
+    "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
+    "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
+    "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
+]
+
+GQA_OK = 0
+GQA_ERR_INVALID_ARGUMENT = 1
+GQA_ERR_UNSUPPORTED = 2
+GQA_ERR_WORKSPACE = 3
+GQA_ERR_CUDA = 4
+GQA_ERR_TIMEOUT = 5
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgqa.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build the CUDA library first "
+        "(python -c 'import __graft_entry__ as g; g.build()'). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_vp, _i32, _ll, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+
+_lib.gqa_attn_fwd.restype = _i32
+_lib.gqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                              _ll, _ll, _ll, _ll, _f32, _vp]
+_lib.gqa_attn_decode_workspace_bytes.restype = _sz
+_lib.gqa_attn_decode_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
+_lib.gqa_attn_decode_num_splits.restype = _i32
+_lib.gqa_attn_decode_num_splits.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
+_lib.gqa_attn_decode.restype = _i32
+_lib.gqa_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                 _ll, _ll, _ll, _ll, _f32, _i32, _vp, _sz, _vp]
+_lib.gqa_status_string.restype = ctypes.c_char_p
+_lib.gqa_status_string.argtypes = [_i32]
+_lib.gqa_get_device_error.restype = _i32
+_lib.gqa_get_device_error.argtypes = [_vp]
+_lib.gqa_selftest_bounded_wait.restype = _i32
+_lib.gqa_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _vp]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+class GqaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {gqa_status_string(status)}" if what else gqa_status_string(status))
+
+
+# ---------------------------------------------------------------- raw C entry points
+def gqa_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                 softmax_scale=0.0, stream=None) -> int:
+    """C ``gqa_attn_fwd``; pointers are integers (device addresses). Returns the status."""
+    return _lib.gqa_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                             float(softmax_scale), stream)
+
+
+def gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits))
+
+
+def gqa_attn_decode_num_splits(B, Hq, Hkv, Tk, D, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_num_splits(B, Hq, Hkv, Tk, D, num_splits))
+
+
+def gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                    softmax_scale=0.0, num_splits=0, workspace=None, workspace_bytes=0,
+                    stream=None) -> int:
+    """C ``gqa_attn_decode``; pointers are integers (device addresses). Returns the status."""
+    return _lib.gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                                float(softmax_scale), num_splits, workspace, workspace_bytes, stream)
+
+
+def gqa_status_string(status: int) -> str:
+    return _lib.gqa_status_string(int(status)).decode()
+
+
+def gqa_get_device_error(stream=None) -> int:
+    return _lib.gqa_get_device_error(stream)
+
+
+def gqa_selftest_bounded_wait(timeout_ns: int, stream=None) -> int:
+    return _lib.gqa_selftest_bounded_wait(int(timeout_ns), stream)
+
+
+# ---------------------------------------------------------------- torch conveniences
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_bf16_cuda(t, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a bf16 CUDA tensor")
+
+
+def _plane_strides(t, name):
+    """(batch, head) element strides of a [B, H, T, D] tensor with packed rows."""
+    if t.dim() != 4 or t.stride(3) != 1 or (t.size(2) > 1 and t.stride(2) != t.size(3)):
+        raise ValueError(f"{name} must be [B, H, T, D] with rows packed (stride(3)=1, stride(2)=D)")
+    return t.stride(0), t.stride(1)
+
+
+def attn_fwd(q, k, v, *, Tk=None, scale=None, return_lse=False, out=None, stream=None):
+    """o = causal GQA attention of q [B,Hq,Tq,D] over k, v [B,Hkv,T_cap,D] (first Tk rows).
+
+    Query row i sits at position Tk - Tq + i. Returns o (bf16, [B,Hq,Tq,D]) and, if
+    ``return_lse``, the fp32 natural-log log-sum-exp [B,Hq,Tq].
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_bf16_cuda(t, n)
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous [B, Hq, Tq, D]")
+    B, Hq, Tq, D = q.shape
+    Hkv = k.shape[1]
+    Tk = k.shape[2] if Tk is None else int(Tk)
+    if k.shape[0] != B or v.shape[:2] != k.shape[:2] or k.shape[3] != D or v.shape[3] != D:
+        raise ValueError("q, k, v shapes disagree")
+    if Tk > k.shape[2] or Tk > v.shape[2]:
+        raise ValueError("Tk exceeds the cache capacity")
+    k_sb, k_sh = _plane_strides(k, "k")
+    v_sb, v_sh = _plane_strides(v, "v")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
+    st = gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Tq, Tk, D,
+                      k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def attn_decode(q, k_cache, v_cache, *, Tk=None, scale=None, num_splits=0, out=None,
+                workspace=None, stream=None):
+    """One decode step: q [B,Hq,1,D] (or [B,Hq,D]) over the first Tk cached keys."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_bf16_cuda(t, n)
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    B, Hq, D = q.shape[0], q.shape[1], q.shape[-1]
+    if q.numel() != B * Hq * D:
+        raise ValueError("decode takes one query per (batch, head)")
+    Hkv = k_cache.shape[1]
+    Tk = k_cache.shape[2] if Tk is None else int(Tk)
+    k_sb, k_sh = _plane_strides(k_cache, "k_cache")
+    v_sb, v_sh = _plane_strides(v_cache, "v_cache")
+    if out is None:
+        out = torch.empty_like(q)
+    need = gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = gqa_attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                         B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh, float(scale or 0.0),
+                         int(num_splits), ws_ptr, ws_bytes, _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_decode")
+    return out

@@ -1,0 +1,426 @@
+// Causal grouped-query attention forward (prefill and suffix chunks) for sm_100a.
+//
+// Computes o_a = softmax(Q_a K_{g(a)}^T * scale + M) V_{g(a)}, g(a) = a / (H_q/H_kv)
+// ("注意力家族", section 统一记号), with the causal mask M placing query row i at
+// absolute position (T_k - T_q) + i ("注意力家族", sections 最小语义实现 and
+// Mask 与增量位置). Execution follows the tiled exact-attention idea ("A Visual
+// Guide to Attention", section "Sources and execution"; "长上下文与高效注意力", the
+// FlashAttention entry): tiles of Q, K and V are staged on chip and merged with an
+// online softmax so the T_q x T_k score matrix never reaches HBM.
+//
+// B200 mapping (one CTA = one work unit = two 128-row query sub-tiles that share
+// every K/V tile):
+//   * warp 0      : TMA producer. Loads both Q sub-tiles once, then K_0, V_0, K_1, V_1 ...
+//                   of KV head g(a) into a ring of 128-key slots (128-byte swizzle).
+//                   K/V are addressed per KV head; nothing is replicated.
+//   * warp 1      : tcgen05 issuer (one thread). S_s = Q_s K_j^T into TMEM (fp32),
+//                   O_s += P_s V_j with P read from TMEM. Completion is signalled with
+//                   tcgen05.commit on mbarriers.
+//   * warp 2      : TMEM allocation (512 columns: S_0, S_1, O_0, O_1).
+//   * warps 4..11 : two softmax warpgroups, one per sub-tile; thread r owns row r
+//                   (TMEM lane r), so row max and row sum need no shuffles. P is
+//                   rounded to bf16 and written over the first half of S in TMEM.
+//                   The running max is refreshed only when it grows by more than
+//                   2^8 (in the log2 domain), so O is rescaled rarely; the final
+//                   O / l and the log-sum-exp are exact whatever max was kept.
+// Causal tile skipping: a sub-tile visits KV tiles 0 .. floor((off + last_row)/128)
+// only, and applies the mask only on tiles that cross its diagonal.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+
+constexpr int kFwdRows = 128;     // query rows per sub-tile (= TMEM lanes)
+constexpr int kFwdKeys = 128;     // keys per KV tile
+constexpr int kFwdThreads = 384;  // 12 warps
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between refreshes
+
+struct FwdParams {
+    int B, Hq, Hkv, Tq, Tk, G;
+    int n_qt;        // ceil(Tq / 128)
+    int pair_heads;  // 1: sub-tiles are heads (a, a+1) of one group on the same rows
+                     // 0: sub-tiles are rows (r, r+128) of one head
+    int per_level;   // work units per row level
+    float scale_log2;
+    __nv_bfloat16* o;
+    float* lse;  // nullable
+    uint32_t* err;
+    unsigned long long timeout_ns;
+};
+
+template <int D>
+struct FwdSmem {
+    static constexpr int kChunks = D / 64;             // 64-element (128-byte) column chunks
+    static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kChunks * kChunkBytes;
+    static constexpr int kStages = D == 128 ? 4 : 8;   // ring slots, each one K or one V tile
+    static constexpr int kQOff = 0;
+    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kCtlOff = kRingOff + kStages * kTileBytes;
+    struct Ctl {
+        uint64_t q_full;
+        uint64_t full[kStages];
+        uint64_t empty[kStages];
+        uint64_t s_full[2];
+        uint64_t p_full[2];
+        uint64_t o_full[2];
+        uint64_t drain;
+        uint32_t tmem_base;
+        uint32_t abort;
+    };
+    static constexpr int kBytes = kCtlOff + (int)sizeof(Ctl) + 1024;  // + alignment slack
+};
+
+struct SubTile {
+    int head;       // query head a
+    int row0;       // first query row of the sub-tile
+    int n_kv;       // KV tiles to visit (0 = sub-tile absent)
+    int masked_from;  // first KV tile that crosses the diagonal
+};
+
+__device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& b, int& g,
+                                                SubTile (&st)[2]) {
+    const int off = p.Tk - p.Tq;
+    const int level = u / p.per_level;
+    const int rest = u - level * p.per_level;
+    if (p.pair_heads) {
+        const int half_g = p.G >> 1;
+        const int rt = p.n_qt - 1 - level;  // longest rows first
+        b = rest / (p.Hkv * half_g);
+        const int hp = rest - b * (p.Hkv * half_g);
+        st[0].head = 2 * hp;
+        st[1].head = 2 * hp + 1;
+        st[0].row0 = st[1].row0 = rt * kFwdRows;
+    } else {
+        const int n_rb = (p.n_qt + 1) >> 1;
+        const int rb = n_rb - 1 - level;
+        b = rest / p.Hq;
+        const int a = rest - b * p.Hq;
+        st[0].head = st[1].head = a;
+        st[0].row0 = rb * 2 * kFwdRows;
+        st[1].row0 = st[0].row0 + kFwdRows;
+    }
+    g = st[0].head / p.G;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        if (st[s].row0 >= p.Tq) {
+            st[s].n_kv = 0;
+            st[s].masked_from = 0;
+        } else {
+            const int last = min(st[s].row0 + kFwdRows - 1, p.Tq - 1);
+            st[s].n_kv = (off + last) / kFwdKeys + 1;
+            st[s].masked_from = (off + st[s].row0 + 1) / kFwdKeys;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    gqa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using L = FwdSmem<D>;
+    using Ctl = typename L::Ctl;
+    constexpr int kStages = L::kStages;
+    constexpr int kTileBytes = L::kTileBytes;
+    constexpr int kChunkBytes = L::kChunkBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t sbase = raw_addr + pad;
+    const uint32_t sQ = sbase + L::kQOff;
+    const uint32_t sRing = sbase + L::kRingOff;
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtlOff);
+    volatile uint32_t* abort_flag = &ctl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    int b, g;
+    SubTile st[2];
+    fwd_decode_unit(p, blockIdx.x, b, g, st);
+    const int n_max = max(st[0].n_kv, st[1].n_kv);
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&ctl->q_full), 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(&ctl->full[i]), 1);
+            mbar_init(smem_u32(&ctl->empty[i]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&ctl->s_full[s]), 1);
+            mbar_init(smem_u32(&ctl->p_full[s]), kFwdRows);
+            mbar_init(smem_u32(&ctl->o_full[s]), 1);
+        }
+        mbar_init(smem_u32(&ctl->drain), 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 32) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const int nq = st[1].n_kv > 0 ? 2 : 1;
+            const uint32_t qbar = smem_u32(&ctl->q_full);
+            mbar_arrive_expect_tx(qbar, nq * kTileBytes);
+            for (int s = 0; s < nq; ++s)
+                for (int c = 0; c < L::kChunks; ++c)
+                    tma_load_4d(sQ + s * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64,
+                                st[s].row0, st[s].head, b);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued[kStages];
+            for (int i = 0; i < kStages; ++i) issued[i] = 0;
+            bool ok = true;
+            for (int j = 0; j < n_max && ok; ++j) {
+                for (int t = 0; t < 2; ++t) {
+                    if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag, p.err,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fbar = smem_u32(&ctl->full[stage]);
+                    mbar_arrive_expect_tx(fbar, kTileBytes);
+                    const CUtensorMap* map = t ? &tm_v : &tm_k;
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
+                                    j * kFwdKeys, g, b);
+                    ++issued[stage];
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag) {
+                // let every copy this thread started land before the CTA exits
+                mbar_wait_drain(qbar, 0, p.timeout_ns);
+                for (int i = 0; i < kStages; ++i)
+                    if (issued[i])
+                        mbar_wait_drain(smem_u32(&ctl->full[i]), (issued[i] - 1u) & 1u, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ tcgen05 issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = umma_idesc_bf16(kFwdRows, kFwdKeys, 0, 0);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16(kFwdRows, D, 0, 1);
+            const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+            const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t pph[2] = {0u, 0u};
+            bool ok = mbar_wait_bounded(smem_u32(&ctl->q_full), 0, abort_flag, p.err, p.timeout_ns);
+
+            auto acquire = [&](int& slot) -> bool {
+                slot = stage;
+                if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), phase, abort_flag, p.err,
+                                       p.timeout_ns))
+                    return false;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                tc_fence_after_sync();
+                return true;
+            };
+            // S_s = Q_s K^T: M=128 rows, N=128 keys, K=D in steps of 16 (32 bytes of a
+            // 128-byte swizzled row; the next 64 columns live in the next chunk).
+            auto issue_qk = [&](int s, int kslot) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+                    const uint64_t a = umma_desc_sw128(sQ + s * kTileBytes + koff, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sRing + kslot * kTileBytes + koff, 16, 1024);
+                    tc_mma_ss(tS[s], a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_s += P_s V: M=128 rows, N=D, K=128 keys in steps of 16. P (bf16, two per
+            // column) sits in the first 64 columns of S_s; V is N-contiguous (d), with
+            // the 64-column chunks LBO apart and 8-key groups 1024 bytes apart.
+            auto issue_pv = [&](int s, int vslot, bool accumulate) {
+#pragma unroll
+                for (int kk = 0; kk < kFwdKeys / 16; ++kk) {
+                    const uint64_t bd =
+                        umma_desc_sw128(sRing + vslot * kTileBytes + kk * 2048, kChunkBytes, 1024);
+                    tc_mma_ts(tO[s], tS[s] + kk * 8, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            int kslot = 0;
+            if (ok && n_max > 0) ok = acquire(kslot);
+            if (ok && n_max > 0) {
+                for (int s = 0; s < 2; ++s)
+                    if (st[s].n_kv > 0) {
+                        issue_qk(s, kslot);
+                        tc_commit(smem_u32(&ctl->s_full[s]));
+                    }
+                tc_commit(smem_u32(&ctl->empty[kslot]));
+            }
+            for (int j = 0; j < n_max && ok; ++j) {
+                int vslot;
+                if (!(ok = acquire(vslot))) break;
+                const bool next = j + 1 < n_max;
+                int knext = -1;
+                for (int s = 0; s < 2 && ok; ++s) {
+                    if (j < st[s].n_kv) {
+                        if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full[s]), pph[s], abort_flag,
+                                                     p.err, p.timeout_ns)))
+                            break;
+                        pph[s] ^= 1u;
+                        tc_fence_after_sync();
+                        issue_pv(s, vslot, j > 0);
+                        if (j == st[s].n_kv - 1) tc_commit(smem_u32(&ctl->o_full[s]));
+                    }
+                    if (s == 1) tc_commit(smem_u32(&ctl->empty[vslot]));
+                    if (next) {
+                        if (knext < 0 && !(ok = acquire(knext))) break;
+                        if (j + 1 < st[s].n_kv) {
+                            issue_qk(s, knext);
+                            tc_commit(smem_u32(&ctl->s_full[s]));
+                        }
+                    }
+                }
+                if (ok && next) tc_commit(smem_u32(&ctl->empty[knext]));
+            }
+            if (*abort_flag) {
+                // wait for the MMAs already issued before TMEM is released
+                tc_commit(smem_u32(&ctl->drain));
+                mbar_wait_drain(smem_u32(&ctl->drain), 0, p.timeout_ns);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int s = (warp - 4) >> 2;
+        const int quad = warp & 3;         // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;    // row within the sub-tile
+        const SubTile me = st[s];
+        if (me.n_kv > 0) {
+            const int off = p.Tk - p.Tq;
+            const int pos = off + me.row0 + r;  // absolute position of this query row
+            const uint32_t lane_sel = (uint32_t)(quad * 32) << 16;
+            const uint32_t tS = tmem + lane_sel + (uint32_t)(s * 128);
+            const uint32_t tO = tmem + lane_sel + 256u + (uint32_t)(s * D);
+            const float sl2 = p.scale_log2;
+            float m = -INFINITY;  // running max of scaled scores (log2 units)
+            float l = 0.f;        // running sum of exp2(score - m)
+            uint32_t sph = 0;
+            bool ok = true;
+            for (int j = 0; j < me.n_kv; ++j) {
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full[s]), sph, abort_flag, p.err,
+                                             p.timeout_ns)))
+                    break;
+                sph ^= 1u;
+                tc_fence_after_sync();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                tc_wait_ld();
+                float tmax = -INFINITY;
+                if (j >= me.masked_from) {
+                    const int lim = pos - j * kFwdKeys;  // columns > lim are in the future
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (c * 32 + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+                        }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(sr[c][e]));
+                const float m_new = fmaxf(m, tmax * sl2);
+                const bool refresh = m_new > m + kRescaleThreshold;
+                float alpha = 1.f;
+                if (refresh) {
+                    alpha = ex2_approx(m - m_new);
+                    l *= alpha;
+                    m = m_new;
+                }
+                if (j > 0 && __any_sync(0xffffffffu, refresh)) {
+                    // O_s has absorbed all earlier P V products (their completion is
+                    // ordered before S_j's commit); rescale this row in place.
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t orr[32];
+                        tmem_ld32(tO + c * 32, orr);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32(tO + c * 32, orr);
+                    }
+                }
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, neg_m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, neg_m));
+                        l += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + c * 16, pk);
+                }
+                tc_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&ctl->p_full[s]));
+            }
+            if (ok && mbar_wait_bounded(smem_u32(&ctl->o_full[s]), 0, abort_flag, p.err, p.timeout_ns)) {
+                tc_fence_after_sync();
+                const int row = me.row0 + r;
+                const float inv_l = 1.f / l;
+                __nv_bfloat16* out =
+                    p.o + (((size_t)b * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + c * 32, orr);
+                    tc_wait_ld();
+                    uint4 v4[4];
+                    uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pw[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
+                                            __uint_as_float(orr[2 * e + 1]) * inv_l);
+                    if (row < p.Tq) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) dst[e] = v4[e];
+                    }
+                }
+                if (p.lse != nullptr && row < p.Tq)
+                    p.lse[((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row] =
+                        (m + __log2f(l)) * 0.69314718055994530942f;
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace gqa

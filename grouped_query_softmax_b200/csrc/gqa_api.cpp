@@ -1,0 +1,210 @@
+// C ABI of libgqa (declared in include/gqa.h): argument checks, TMA descriptor
+// encoding, split planning and dispatch to the kernel launchers. No device memory is
+// allocated here and no state is kept between calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "../../include/gqa.h"
+#include "../../include/gqa_testing.h"
+#include "gqa_internal.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A [B, H, T, D] bf16 view with packed rows and free (b, h) strides, tiled as boxes of
+// 128 rows x 64 columns (128 bytes) with the 128-byte swizzle. Strides in elements.
+gqa_status make_map(CUtensorMap* map, const void* base, int B, int H, int T, int D,
+                    long long s_b, long long s_h) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GQA_ERR_CUDA;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)s_h * 2, (cuuint64_t)s_b * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)gqa::kTileRows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_UNSUPPORTED;
+}
+
+// Strides of a dimension of extent 1 are never used; give TMA a harmless legal value.
+long long effective_stride(long long s, int extent, long long fallback) {
+    return extent == 1 ? fallback : s;
+}
+
+gqa_status check_kv_strides(int B, int Hkv, int Tk, int D, long long& sb, long long& sh) {
+    const long long plane = (long long)Tk * D;
+    sh = effective_stride(sh, Hkv, plane);
+    sb = effective_stride(sb, B, plane * Hkv);
+    if (sb <= 0 || sh <= 0) return GQA_ERR_INVALID_ARGUMENT;
+    if ((sb & 7) || (sh & 7)) return GQA_ERR_INVALID_ARGUMENT;  // 16-byte TMA strides
+    if (sb * 2 >= (1LL << 40) || sh * 2 >= (1LL << 40)) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+gqa_status check_common(int B, int Hq, int Hkv, int Tq, int Tk, int D) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || D <= 0) return GQA_ERR_INVALID_ARGUMENT;
+    if (Hq % Hkv != 0 || Tq > Tk) return GQA_ERR_INVALID_ARGUMENT;
+    if (D != 64 && D != 128) return GQA_ERR_UNSUPPORTED;
+    // flat element offsets of q and o must fit in 63 bits; grid and TMA limits below
+    if ((long long)B * Hq > (1LL << 30)) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    return sms;
+}
+
+struct SplitPlan {
+    int splits, blk_per_split, n_blk;
+};
+
+SplitPlan plan_splits(int B, int Hq, int Hkv, int Tk, int requested) {
+    SplitPlan sp{};
+    sp.n_blk = (Tk + gqa::kTileKeys - 1) / gqa::kTileKeys;
+    const int G = Hq / Hkv;
+    const long long units = (long long)B * Hkv * ((G + 15) / 16);
+    int want = requested;
+    if (want <= 0) {
+        // about four waves of one CTA per SM, each split at least 8 tiles (1024 keys)
+        const long long target = 4LL * device_sm_count();
+        want = (int)std::min<long long>((target + units - 1) / units, 1 << 20);
+        want = std::min(want, std::max(1, sp.n_blk / 8));
+    }
+    want = std::max(1, std::min(want, sp.n_blk));
+    sp.blk_per_split = (sp.n_blk + want - 1) / want;
+    sp.splits = (sp.n_blk + sp.blk_per_split - 1) / sp.blk_per_split;  // no empty split
+    return sp;
+}
+
+size_t ws_lse_offset(int splits, int B, int Hq, int D) {
+    const size_t o_bytes = (size_t)splits * B * Hq * D * sizeof(float);
+    return (o_bytes + 255) & ~(size_t)255;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_status_string(gqa_status s) {
+    switch (s) {
+        case GQA_OK: return "GQA_OK";
+        case GQA_ERR_INVALID_ARGUMENT: return "GQA_ERR_INVALID_ARGUMENT";
+        case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED";
+        case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE";
+        case GQA_ERR_CUDA: return "GQA_ERR_CUDA";
+        case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT";
+    }
+    return "GQA_ERR_UNKNOWN";
+}
+
+gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh,
+                        long long v_sb, long long v_sh, float softmax_scale, void* stream) {
+    gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GQA_ERR_INVALID_ARGUMENT;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+
+    gqa::FwdLaunch a{};
+    const long long q_sh = (long long)Tq * D;
+    if ((st = make_map(&a.tm_q, q, B, Hq, Tq, D, q_sh * Hq, q_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.o = o;
+    a.lse = lse;
+    return gqa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
+    if (check_common(B, Hq, Hkv, 1, Tk, D) != GQA_OK) return 0;
+    return plan_splits(B, Hq, Hkv, Tk, num_splits).splits;
+}
+
+size_t gqa_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
+    if (check_common(B, Hq, Hkv, 1, Tk, D) != GQA_OK) return 0;
+    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tk, num_splits);
+    if (sp.splits == 1) return 0;
+    return ws_lse_offset(sp.splits, B, Hq, D) + (size_t)sp.splits * B * Hq * sizeof(float);
+}
+
+gqa_status gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, int B,
+                           int Hq, int Hkv, int Tk, int D, long long k_sb, long long k_sh,
+                           long long v_sb, long long v_sh, float softmax_scale, int num_splits,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    gqa_status st = check_common(B, Hq, Hkv, 1, Tk, D);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+        return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tk, num_splits);
+    gqa::DecLaunch a{};
+    if (sp.splits > 1) {
+        const size_t need = ws_lse_offset(sp.splits, B, Hq, D) + (size_t)sp.splits * B * Hq * sizeof(float);
+        if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return GQA_ERR_WORKSPACE;
+        a.ws_o = static_cast<float*>(workspace);
+        a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_lse_offset(sp.splits, B, Hq, D));
+    }
+    if ((st = make_map(&a.tm_k, k_cache, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_v, v_cache, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tk = Tk; a.D = D;
+    a.splits = sp.splits;
+    a.blk_per_split = sp.blk_per_split;
+    a.n_blk = sp.n_blk;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.q = q;
+    a.o = o;
+    return gqa::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+gqa_status gqa_get_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+    uint32_t v = 0;
+    if (gqa::read_and_clear_device_error(&v) != cudaSuccess) return GQA_ERR_CUDA;
+    return v ? GQA_ERR_TIMEOUT : GQA_OK;
+}
+
+gqa_status gqa_selftest_bounded_wait(unsigned long long timeout_ns, void* stream) {
+    if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return GQA_ERR_INVALID_ARGUMENT;
+    return gqa::launch_selftest_wait(timeout_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+// Kernel translation unit: every device kernel of libgqa and its launcher.
+// Keeping them in one unit lets them share one device error word without
+// relocatable device code.
+#include <cuda_runtime.h>
+
+#include "decode_sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "gqa_internal.h"
+
+namespace gqa {
+
+// Bit flags (kDevErr*) set by bounded waits that ran out; see gqa_get_device_error().
+__device__ uint32_t g_device_error = 0;
+
+static uint32_t* device_error_ptr() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    return static_cast<uint32_t*>(p);
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
+    FwdParams p{};
+    p.B = a.B;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.Tq = a.Tq;
+    p.Tk = a.Tk;
+    p.G = a.Hq / a.Hkv;
+    p.n_qt = (a.Tq + kFwdRows - 1) / kFwdRows;
+    p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+    long long units;
+    if (p.pair_heads) {
+        p.per_level = a.B * a.Hkv * (p.G / 2);
+        units = (long long)p.per_level * p.n_qt;
+    } else {
+        p.per_level = a.B * a.Hq;
+        units = (long long)p.per_level * ((p.n_qt + 1) / 2);
+    }
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.o = static_cast<__nv_bfloat16*>(a.o);
+    p.lse = a.lse;
+    p.err = device_error_ptr();
+    p.timeout_ns = kWaitTimeoutNs;
+    if (!p.err) return cudaErrorUnknown;
+    if (units <= 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int smem = FwdSmem<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    gqa_fwd_sm100_kernel<D><<<(unsigned)units, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdLaunch& a, cudaStream_t stream) {
+    return a.D == 128 ? launch_fwd_d<128>(a, stream) : launch_fwd_d<64>(a, stream);
+}
+
+template <int D>
+static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
+    DecParams p{};
+    p.B = a.B;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.Tk = a.Tk;
+    p.G = a.Hq / a.Hkv;
+    p.n_hc = (p.G + kDecRows - 1) / kDecRows;
+    p.splits = a.splits;
+    p.blk_per_split = a.blk_per_split;
+    p.n_blk = a.n_blk;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.q = static_cast<const __nv_bfloat16*>(a.q);
+    p.o = static_cast<__nv_bfloat16*>(a.o);
+    p.ws_o = a.ws_o;
+    p.ws_lse = a.ws_lse;
+    p.err = device_error_ptr();
+    p.timeout_ns = kWaitTimeoutNs;
+    if (!p.err) return cudaErrorUnknown;
+    const int smem = DecSmem<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(gqa_decode_sm100_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.splits, (unsigned)(a.Hkv * p.n_hc), (unsigned)a.B);
+    gqa_decode_sm100_kernel<D><<<grid, kDecThreads, smem, stream>>>(a.tm_k, a.tm_v, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.splits == 1) return e;
+    const int rows = a.B * a.Hq;
+    gqa_decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        a.ws_o, a.ws_lse, static_cast<__nv_bfloat16*>(a.o), rows, a.splits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream) {
+    return a.D == 128 ? launch_decode_d<128>(a, stream) : launch_decode_d<64>(a, stream);
+}
+
+// One CTA, one thread: wait on an mbarrier that never completes, bounded by
+// timeout_ns, through the same routine the production kernels use.
+__global__ void gqa_selftest_wait_kernel(uint32_t* err, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // phase 0 never completes: nothing arrives on the barrier
+        (void)mbar_wait_bounded(smem_u32(&bar), 0, &abort_flag, err, timeout_ns);
+    }
+}
+
+cudaError_t launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream) {
+    uint32_t* err = device_error_ptr();
+    if (!err) return cudaErrorUnknown;
+    gqa_selftest_wait_kernel<<<1, 32, 0, stream>>>(err, timeout_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(uint32_t* value) {
+    uint32_t zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    if (*value) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
+    return e;
+}
+
+}  // namespace gqa

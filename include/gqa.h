@@ -1,0 +1,124 @@
+/*
+ * gqa.h -- C ABI of libgqa: causal grouped-query softmax attention on B200 (sm_100a).
+ *
+ * The operation (one definition covers MHA, GQA and MQA):
+ *
+ *   o_a = softmax( Q_a K_{g(a)}^T * scale + M ) V_{g(a)},   g(a) = floor(a / (H_q / H_kv))
+ *
+ *   -- "注意力家族" (wineandchord.com, attention variants), section 统一记号 (the o_a
+ *      equation) and section 最小语义实现 (interface q:[B,H_q,T_q,D], k,v:[B,H_kv,T_k,D];
+ *      consecutive H_q/H_kv query heads map to one KV head; H_q % H_kv == 0 and
+ *      T_q <= T_k are required; scale 1/sqrt(D); the result has q's dtype).
+ *   -- "Attention Architecture Evolution", section GQA (group(i) = floor(i/(Hq/Hkv))).
+ *
+ * M is the causal mask with the suffix offset: query row i (0 <= i < T_q) sits at
+ * absolute position (T_k - T_q) + i and sees keys j <= (T_k - T_q) + i, its own
+ * position included ("注意力家族", sections 最小语义实现 and Mask 与增量位置; "A Visual
+ * Guide to Attention", section "Which positions are visible?"). There is no
+ * non-causal mode.
+ *
+ * Types and precision: Q, K, V and O are bf16; products accumulate in fp32; the
+ * softmax runs in fp32 and its probabilities are rounded to bf16 before the product
+ * with V (the pages' reference rounds the fp32 probabilities to the input dtype
+ * before "@ v"); O is rounded to bf16 round-to-nearest-even.
+ *
+ * Memory: every pointer is a DEVICE pointer owned by the caller. The library never
+ * allocates device memory and keeps no per-call state; K and V are addressed per KV
+ * head and are never replicated per query head. All calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream) and return as soon as
+ * the kernels are enqueued. Calls are thread-safe and re-entrant.
+ *
+ * Errors: argument checks run on the host before anything is enqueued; a call that
+ * returns an error has launched nothing. Launch failures return GQA_ERR_CUDA.
+ * Device-side waits are bounded; a wait that runs out sets a device error word
+ * that gqa_get_device_error() reports as GQA_ERR_TIMEOUT.
+ */
+#ifndef GQA_H_
+#define GQA_H_
+
+#include <stddef.h>
+
+/* Symbols of the C ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gqa_status {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size or stride, Hq % Hkv, Tq > Tk */
+    GQA_ERR_UNSUPPORTED = 2,      /* D not in {64, 128}, sizes beyond grid or TMA limits */
+    GQA_ERR_WORKSPACE = 3,        /* decode workspace missing or smaller than required */
+    GQA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or a kernel launch failed */
+    GQA_ERR_TIMEOUT = 5           /* a bounded device-side wait ran out (reported later) */
+} gqa_status;
+
+/*
+ * Prefill and suffix chunks (1 <= T_q <= T_k).
+ *
+ *   q    bf16 [B, Hq, Tq, D], contiguous; 16-byte aligned.
+ *   k    bf16; element (b, h, t, d) at k + b*k_sb + h*k_sh + t*D + d (elements).
+ *        Rows are packed (row stride D); batch/head strides are free, so a cache
+ *        pre-allocated to a capacity T_cap >= T_k is read as its [:T_k] slice.
+ *        16-byte aligned; k_sb and k_sh multiples of 8 elements.
+ *   v    bf16; same addressing with v_sb, v_sh.
+ *   o    bf16 [B, Hq, Tq, D], contiguous; written. Must not overlap the inputs.
+ *   lse  fp32 [B, Hq, Tq] or NULL; if given, receives the natural-log
+ *        log-sum-exp of each row's scaled, masked scores.
+ *   softmax_scale  <= 0 selects 1/sqrt(D).
+ *   D    64 or 128.
+ */
+GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int Tq, int Tk, int D,
+                        long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                        float softmax_scale, void* stream);
+
+/*
+ * Decode (T_q = 1): the query of each (b, a) sits at position T_k - 1 and sees all
+ * T_k cached keys ("注意力家族", section 最小语义实现: the suffix case with one
+ * query). The KV cache is split into num_splits key ranges; each range yields a
+ * partial result (fp32 output and log-sum-exp) and a second kernel merges them in
+ * fixed split order, so the result is deterministic.
+ *
+ *   q        bf16 [B, Hq, 1, D], contiguous; 16-byte aligned.
+ *   k_cache, v_cache  addressed as k/v of gqa_attn_fwd, first T_k rows read.
+ *   o        bf16 [B, Hq, 1, D], contiguous; written.
+ *   num_splits  0 = choose automatically; otherwise the requested split count
+ *            (clamped to [1, ceil(T_k / 128)]).
+ *   workspace   device buffer of at least gqa_attn_decode_workspace_bytes(...)
+ *            bytes (same arguments), 256-byte aligned; may be NULL when that size
+ *            is 0 (a single split writes o directly). Its contents on entry are
+ *            ignored; it must not be shared by calls that can overlap on the GPU.
+ */
+GQA_API size_t gqa_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Tk, int D, int num_splits);
+
+GQA_API gqa_status gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                           int B, int Hq, int Hkv, int Tk, int D,
+                           long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                           float softmax_scale, int num_splits,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* The split count gqa_attn_decode will use for these arguments (num_splits 0 = auto). */
+GQA_API int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits);
+
+/* A static, human-readable name for a status code. */
+GQA_API const char* gqa_status_string(gqa_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device. Returns GQA_ERR_TIMEOUT if a bounded wait in any kernel of this
+ * library ran out since the last call, GQA_ERR_CUDA if the stream reports a CUDA
+ * error, else GQA_OK.
+ */
+GQA_API gqa_status gqa_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H_ */

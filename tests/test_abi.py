@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    import grouped_query_softmax_b200 as m
+    return m
+
+
+def declared_functions():
+    names = []
+    for h in ("gqa.h", "gqa_testing.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(gqa_[a-z_0-9]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(gqa):
+    lib = ctypes.CDLL(gqa.library_path())
+    names = declared_functions()
+    assert {"gqa_attn_fwd", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
+            "gqa_status_string", "gqa_get_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared but not exported"
+
+
+def test_only_declared_symbols_are_exported(gqa):
+    out = os.popen(f"nm -D --defined-only {gqa.library_path()}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("gqa")}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(gqa):
+    assert gqa.gqa_status_string(gqa.GQA_OK) == "GQA_OK"
+    assert gqa.gqa_status_string(gqa.GQA_ERR_TIMEOUT) == "GQA_ERR_TIMEOUT"
+    assert gqa.gqa_status_string(99) == "GQA_ERR_UNKNOWN"
+
+
+P = 1 << 20  # a 16-byte-aligned fake device address; never dereferenced on these paths
+
+
+def fwd(gqa, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=None, B=1, Hq=4, Hkv=2, Tq=8, Tk=8, D=64,
+             k_sb=2 * 8 * 64, k_sh=8 * 64, v_sb=2 * 8 * 64, v_sh=8 * 64, softmax_scale=0.0, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_fwd(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(k=P + 8), 1),       # null / misaligned
+    (dict(Hq=3), 1),                                                   # Hq % Hkv != 0
+    (dict(Tq=9), 1),                                                   # Tq > Tk
+    (dict(B=0), 1), (dict(Tk=0, Tq=0), 1), (dict(Hkv=0), 1),
+    (dict(D=96), 2), (dict(D=256), 2),                                # unsupported head dim
+    (dict(k_sh=8 * 64 + 4), 1), (dict(B=2, v_sb=-512), 1),            # bad strides (a batch stride of B=1 is unused)
+    (dict(softmax_scale=float("nan")), 1),
+    (dict(lse=P + 2), 1),
+])
+def test_fwd_rejects_bad_arguments(gqa, kw, status):
+    assert fwd(gqa, **kw) == status
+
+
+def dec(gqa, **kw):
+    a = dict(q=P, k_cache=P, v_cache=P, o=P, B=1, Hq=4, Hkv=2, Tk=1024, D=128,
+             k_sb=2 * 1024 * 128, k_sh=1024 * 128, v_sb=2 * 1024 * 128, v_sh=1024 * 128,
+             softmax_scale=0.0, num_splits=4, workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_decode(**a)
+
+
+def test_decode_rejects_bad_arguments_and_small_workspace(gqa):
+    assert dec(gqa, Hq=6, Hkv=4) == gqa.GQA_ERR_INVALID_ARGUMENT
+    assert dec(gqa, D=80) == gqa.GQA_ERR_UNSUPPORTED
+    assert dec(gqa, q=None) == gqa.GQA_ERR_INVALID_ARGUMENT
+    need = gqa.gqa_attn_decode_workspace_bytes(1, 4, 2, 1024, 128, 4)
+    assert need > 0
+    assert dec(gqa) == gqa.GQA_ERR_WORKSPACE                          # none given
+    assert dec(gqa, workspace=P, workspace_bytes=need - 4) == gqa.GQA_ERR_WORKSPACE
+    assert dec(gqa, workspace=P + 16, workspace_bytes=need) == gqa.GQA_ERR_WORKSPACE  # not 256-aligned
+
+
+def test_decode_split_planning(gqa):
+    # explicit requests are clamped to [1, ceil(Tk/128)] and never leave a split empty
+    assert gqa.gqa_attn_decode_num_splits(1, 4, 2, 1024, 128, 4) == 4
+    assert gqa.gqa_attn_decode_num_splits(1, 4, 2, 1024, 128, 100) == 8
+    assert gqa.gqa_attn_decode_num_splits(1, 4, 2, 1100, 128, 4) == 3   # 9 tiles -> 3 per split
+    assert gqa.gqa_attn_decode_num_splits(1, 4, 2, 100, 128, 0) == 1
+    assert gqa.gqa_attn_decode_workspace_bytes(1, 4, 2, 1024, 128, 1) == 0
+    s = 4
+    o_bytes = s * 1 * 4 * 128 * 4
+    assert gqa.gqa_attn_decode_workspace_bytes(1, 4, 2, 1024, 128, s) == ((o_bytes + 255) // 256) * 256 + s * 4 * 4
+
+
+def test_selftest_rejects_out_of_range_timeouts(gqa):
+    assert gqa.gqa_selftest_bounded_wait(10) == gqa.GQA_ERR_INVALID_ARGUMENT
+    assert gqa.gqa_selftest_bounded_wait(10 ** 11) == gqa.GQA_ERR_INVALID_ARGUMENT
+
+
+def test_product_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "grouped_query_softmax_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".cpp", ".h")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in txt and "gqa_oracle" not in txt, f
