@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of causal grouped-query softmax attention on B200.
+
+One step = one pass of the hot path over one batch of synthetic input:
+  * headline: gqa_attn_fwd on the GQA prefill workload (B4 Hq32 Hkv8 T4096 D128),
+    metric TFLOP/s with FLOPs = 4 * D * Hq * B * (causal-visible query/key pairs);
+  * "decode" object: gqa_attn_decode on the GQA decode workload (B64 Hq32 Hkv8,
+    T_k 32768, D128), metric KV GB/s = (K + V bytes) / time.
+Inputs are seeded iid N(0,1) rounded to bf16 (see gqa_inputs), resident in HBM
+when the timed region starts. Under torchrun every rank runs its own copy of the
+workload (independent problems, no data-path collective): weak scaling, value =
+all ranks' work / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of the
+method here) on a bounded row sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import gqa_inputs as gi  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["grouped_query_softmax_b200/csrc/fwd_sm100.cuh",
+                  "grouped_query_softmax_b200/csrc/decode_sm100.cuh",
+                  "grouped_query_softmax_b200/csrc/sm100_ptx.cuh"]
+
+
+# ---------------------------------------------------------------- work counts
+def visible_pairs(Tq: int, Tk: int) -> int:
+    """Causal-visible (query, key) pairs per (b, a): row i sees Tk - Tq + i + 1 keys."""
+    return Tq * (Tk - Tq) + Tq * (Tq + 1) // 2
+
+
+def algorithmic_flops(w) -> float:
+    return 4.0 * w.D * w.Hq * w.B * visible_pairs(w.Tq, w.Tk)
+
+
+def kv_bytes(w) -> int:
+    return 2 * w.B * w.Hkv * w.Tk * w.D * 2
+
+
+def qo_bytes(w) -> int:
+    return 2 * w.B * w.Hq * w.Tq * w.D * 2
+
+
+def row_flops(w, rows) -> float:
+    i = np.asarray(rows) % w.Tq
+    return float(np.sum(4.0 * w.D * (w.Tk - w.Tq + i + 1)))
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel sources still
+    match the ones that capture was taken with; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the GPU is busy."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.gpu_id is not None:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._reader, daemon=True).start()
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        window = [s for t, s in self.samples if t0 <= t <= t1]
+        scope = "timed region"
+        if len(window) < 3:
+            window = [s for _, s in self.samples]
+            scope = "whole run (timed region shorter than the sampling interval)"
+        if not window:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "scope": "unavailable"}
+        sm = [num(s[1]) for s in window if num(s[1]) is not None]
+        smax = [num(s[2]) for s in window if num(s[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in window for i in range(4) if s[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(window), "scope": scope}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- GPU measurements
+def to_device(arr_u16, dev):
+    import torch
+    return torch.from_numpy(arr_u16.view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def timed(fn, steps, warmup, world, dev):
+    """Run fn() warmup times, then time exactly `steps` calls on the current stream.
+    Returns (max-over-ranks ms for the whole timed region, t_start, t_end wall)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    return max_over_ranks(ms, world, dev), t0, t1
+
+
+def measure_prefill(w, steps, warmup, world, dev, e2e_steps):
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, k, v = w.make()
+    qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
+    od = torch.empty_like(qd)
+    fn = lambda: gqa.attn_fwd(qd, kd, vd, out=od)
+    ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after prefill timing: {gqa.gqa_status_string(st)}")
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": steps}
+
+    # end to end through the public API: pinned host inputs in, host output out, every step
+    qh = torch.from_numpy(q.view(np.int16)).pin_memory()
+    kh = torch.from_numpy(k.view(np.int16)).pin_memory()
+    vh = torch.from_numpy(v.view(np.int16)).pin_memory()
+    oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+    qi, ki, vi, oi = (x.view(torch.int16) for x in (qd, kd, vd, od))
+
+    def e2e_step():
+        qi.copy_(qh, non_blocking=True)
+        ki.copy_(kh, non_blocking=True)
+        vi.copy_(vh, non_blocking=True)
+        gqa.attn_fwd(qd, kd, vd, out=od)
+        oh.copy_(oi, non_blocking=True)
+    e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
+    res["e2e_ms_total"] = e2e_ms
+    res["e2e_steps"] = e2e_steps
+    res["h2d_bytes"] = int(q.nbytes + k.nbytes + v.nbytes)
+    res["d2h_bytes"] = int(q.nbytes)
+    del qd, kd, vd, od
+    return res
+
+
+def measure_decode(w, steps, warmup, world, dev, e2e_steps):
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, k, v = w.make()
+    qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
+    od = torch.empty_like(qd)
+    splits = gqa.gqa_attn_decode_num_splits(w.B, w.Hq, w.Hkv, w.Tk, w.D, 0)
+    need = gqa.gqa_attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Tk, w.D, 0)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    fn = lambda: gqa.attn_decode(qd, kd, vd, out=od, workspace=ws)
+    ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after decode timing: {gqa.gqa_status_string(st)}")
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "splits": splits,
+           "launches": steps * (1 if splits == 1 else 2)}
+    qh = torch.from_numpy(q.view(np.int16)).pin_memory()
+    kh = torch.from_numpy(k.view(np.int16)).pin_memory()
+    vh = torch.from_numpy(v.view(np.int16)).pin_memory()
+    oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+    qi, ki, vi, oi = (x.view(torch.int16) for x in (qd, kd, vd, od))
+
+    def e2e_step():
+        qi.copy_(qh, non_blocking=True)
+        ki.copy_(kh, non_blocking=True)
+        vi.copy_(vh, non_blocking=True)
+        gqa.attn_decode(qd, kd, vd, out=od, workspace=ws)
+        oh.copy_(oi, non_blocking=True)
+    e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
+    res.update(e2e_ms_total=e2e_ms, e2e_steps=e2e_steps, h2d_bytes=int(q.nbytes + k.nbytes + v.nbytes),
+               d2h_bytes=int(q.nbytes))
+    del qd, kd, vd, od, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- the oracle on the host
+def oracle_sample(w, budget_s: float, threads: int, q=None, k=None, v=None):
+    """Time the fp64 oracle on a seeded row sample sized to about budget_s seconds.
+    Returns (flops_done, seconds, rows)."""
+    import oracle
+    if q is None:
+        q, k, v = w.make()
+    rng = np.random.default_rng(0)
+    total = w.B * w.Hq * w.Tq
+    probe = rng.integers(0, total, size=min(total, max(threads, 16)))
+    t = time.perf_counter()
+    oracle.attention_rows(q, k, v, probe, threads=threads)
+    dt = max(time.perf_counter() - t, 1e-6)
+    rate = row_flops(w, probe) / dt
+    mean_row = row_flops(w, np.arange(total)) / total if total <= 1 << 22 else 4.0 * w.D * (
+        w.Tk - w.Tq + w.Tq / 2)
+    n = int(min(total, max(threads, budget_s * rate / mean_row)))
+    rows = np.sort(rng.choice(total, size=n, replace=False)) if n < total else np.arange(total)
+    t = time.perf_counter()
+    oracle.attention_rows(q, k, v, rows, threads=threads)
+    dt = time.perf_counter() - t
+    return row_flops(w, rows), dt, rows
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- main
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa_prefill", choices=sorted(gi.WORKLOADS))
+    ap.add_argument("--decode-workload", default="gqa_decode", choices=sorted(gi.WORKLOADS))
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args(argv)
+
+
+def workload_config(w, extra=None):
+    c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Tq": w.Tq, "Tk": w.Tk, "D": w.D,
+         "q_scale": 2 ** w.q_pow2, "seed": w.seed, "causal": True}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def metric_of(w):
+    if w.Tq == 1:
+        return "GQA attn KV GB/s (decode) on 1 B200, % of roofline", "GB/s"
+    return "GQA attn TFLOP/s (prefill) on 1 B200, % of roofline", "TFLOP/s"
+
+
+def throughput(w, ms_per_step, world):
+    if w.Tq == 1:
+        return world * kv_bytes(w) / (ms_per_step * 1e-3) / 1e9
+    return world * algorithmic_flops(w) / (ms_per_step * 1e-3) / 1e12
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference arm: rank 0 alone runs it; other ranks exit 0."""
+    if rank != 0:
+        return
+    w = gi.WORKLOADS[args.workload]
+    threads = cpu_threads()
+    q, k, v = w.make()
+    per_step_budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step_budget, threads, q, k, v)
+    flops = secs = 0.0
+    rows_total = 0
+    for _ in range(args.steps):
+        f, s, rows = oracle_sample(w, per_step_budget, threads, q, k, v)
+        flops += f
+        secs += s
+        rows_total += len(rows)
+    metric, unit = metric_of(w)
+    if w.Tq == 1:
+        frac = rows_total / (args.steps * w.B * w.Hq)
+        value = frac * kv_bytes(w) * args.steps / secs / 1e9
+    else:
+        value = flops / secs / 1e12
+    sample = f"{rows_total} output rows in {args.steps} steps (row-sampled, fp64, {per_step_budget:.1f} s per step)"
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus > 1 needs torchrun (one process per GPU)")
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    import grouped_query_softmax_b200 as gqa  # noqa: F401  (fails loudly without libgqa.so)
+
+    peaks, peak_src = load_peaks()
+    w = gi.WORKLOADS[args.workload]
+    gpu_id = None
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        gpu_id = vis.split(",")[local]
+    elif world > 1:
+        gpu_id = str(local)
+    sampler = ClockSampler(gpu_id if gpu_id is not None else "0")
+    sampler.start()
+    time.sleep(0.2)
+
+    metric, unit = metric_of(w)
+    if w.Tq == 1:
+        r = measure_decode(w, args.steps, args.warmup, world, dev, args.e2e_steps)
+    else:
+        r = measure_prefill(w, args.steps, args.warmup, world, dev, args.e2e_steps)
+    ms_step = r["ms_total"] / args.steps
+    value = throughput(w, ms_step, world)
+    e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
+    clocks = sampler.summary(r["t0"], r["t1"])
+
+    if w.Tq == 1:
+        per_launch_bytes = kv_bytes(w) + qo_bytes(w)
+        achieved = per_launch_bytes / (ms_step * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": load_traffic("gqa_decode_sm100_kernel", w.name),
+                "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)",
+                "kernel": "gqa_decode_sm100_kernel + gqa_decode_combine_kernel (one call per step)"}
+    else:
+        achieved = algorithmic_flops(w) / (ms_step * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": load_traffic("gqa_fwd_sm100_kernel", w.name),
+                "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed alone)",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "frac_of_spec_2250": achieved / 2250.0,
+                "kernel": "gqa_fwd_sm100_kernel"}
+
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, {"l2": "inputs larger than L2 (no flush)",
+                                          "parallelism": f"dp{world} (independent problems per rank)"}),
+            "roofline": roof,
+            "e2e": {"value": throughput(w, e2e_ms, world), "unit": unit,
+                    "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"],
+                    "ms_per_step": e2e_ms, "steps": r["e2e_steps"]},
+            "gpu_launches": r["launches"], "clocks": clocks}
+
+    if not args.no_decode and w.Tq != 1:
+        wd = gi.WORKLOADS[args.decode_workload]
+        rd = measure_decode(wd, max(3, args.steps // 20), max(3, args.warmup), world, dev,
+                            max(2, args.e2e_steps // 5))
+        msd = rd["ms_total"] / max(3, args.steps // 20)
+        gbs = throughput(wd, msd, world)
+        ach = (kv_bytes(wd) + qo_bytes(wd)) / (msd * 1e-3) / 1e9
+        line["decode"] = {
+            "metric": "KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": msd,
+            "steps": max(3, args.steps // 20), "config": workload_config(wd, {"splits": rd["splits"]}),
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"],
+                         "traffic": load_traffic("gqa_decode_sm100_kernel", wd.name),
+                         "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
+            "e2e": {"value": throughput(wd, rd["e2e_ms_total"] / rd["e2e_steps"], world), "unit": "GB/s",
+                    "h2d_bytes_per_step": rd["h2d_bytes"], "d2h_bytes_per_step": rd["d2h_bytes"]},
+            "gpu_launches": rd["launches"]}
+    sampler.stop()
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        threads = cpu_threads()
+        flops, secs, rows = oracle_sample(w, args.cpu_budget, threads)
+        if w.Tq == 1:
+            cv = len(rows) / (w.B * w.Hq) * kv_bytes(w) / secs / 1e9
+        else:
+            cv = flops / secs / 1e12
+        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": threads, "kind": "oracle",
+                                "sample": f"{len(rows)} of {w.B * w.Hq * w.Tq} output rows "
+                                          f"(seeded sample, fp64), {secs:.1f} s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

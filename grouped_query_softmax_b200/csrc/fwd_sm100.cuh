@@ -8,9 +8,10 @@
 // FlashAttention entry): tiles of Q, K and V are staged on chip and merged with an
 // online softmax so the T_q x T_k score matrix never reaches HBM.
 //
-// B200 mapping (one CTA = one work unit = two 128-row query sub-tiles that share
-// every K/V tile):
-//   * warp 0      : TMA producer. Loads both Q sub-tiles once, then K_0, V_0, K_1, V_1 ...
+// B200 mapping: a work unit is two 128-row query sub-tiles that share every K/V tile;
+// units are ordered longest first and a persistent CTA per SM strides over them, so
+// the next unit's Q load and Q K^T products overlap the current unit's epilogue.
+//   * warp 0      : TMA producer. Loads both Q sub-tiles of a unit, then K_0, V_0, K_1, V_1 ...
 //                   of KV head g(a) into a ring of 128-key slots (128-byte swizzle).
 //                   K/V are addressed per KV head; nothing is replicated.
 //   * warp 1      : tcgen05 issuer (one thread). S_s = Q_s K_j^T into TMEM (fp32),
@@ -27,14 +28,29 @@
 // only, and applies the mask only on tiles that cross its diagonal.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace gqa {
 
 constexpr int kFwdRows = 128;     // query rows per sub-tile (= TMEM lanes)
 constexpr int kFwdKeys = 128;     // keys per KV tile
-constexpr int kFwdThreads = 384;  // 12 warps
+constexpr int kFwdThreads = 384;  // 12 warps = 3 warpgroups
+// Register split (setmaxnreg): the launch gives 384 threads x kFwdLaunchRegs; the
+// producer/MMA warpgroup drops to kFwdCtlRegs so the two softmax warpgroups can hold
+// a full 128-column score row without spilling. 128 * (104 + 200 + 200) = 384 * 168.
+constexpr int kFwdLaunchRegs = 168;
+constexpr int kFwdCtlRegs = 104;
+constexpr int kFwdSoftmaxRegs = 200;
+static_assert(128 * (kFwdCtlRegs + 2 * kFwdSoftmaxRegs) <= kFwdThreads * kFwdLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between refreshes
+#ifndef GQA_FWD_POLY_EVERY
+#define GQA_FWD_POLY_EVERY 0
+#endif
+// every kPolyEvery-th column pair of an unmasked tile takes the polynomial exp2 (0 = none)
+constexpr int kPolyEvery = GQA_FWD_POLY_EVERY;
 
 struct FwdParams {
     int B, Hq, Hkv, Tq, Tk, G;
@@ -42,6 +58,7 @@ struct FwdParams {
     int pair_heads;  // 1: sub-tiles are heads (a, a+1) of one group on the same rows
                      // 0: sub-tiles are rows (r, r+128) of one head
     int per_level;   // work units per row level
+    int units;       // total work units (grid-strided by the persistent CTAs)
     float scale_log2;
     __nv_bfloat16* o;
     float* lse;  // nullable
@@ -60,11 +77,13 @@ struct FwdSmem {
     static constexpr int kCtlOff = kRingOff + kStages * kTileBytes;
     struct Ctl {
         uint64_t q_full;
+        uint64_t q_empty;
         uint64_t full[kStages];
         uint64_t empty[kStages];
         uint64_t s_full[2];
         uint64_t p_full[2];
         uint64_t o_full[2];
+        uint64_t o_empty[2];
         uint64_t drain;
         uint32_t tmem_base;
         uint32_t abort;
@@ -115,6 +134,12 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
     }
 }
 
+// k-th unit of persistent CTA i out of n: a boustrophedon walk over the longest-first
+// unit list (i, 2n-1-i, 2n+i, ...), so each CTA's total work is nearly equal.
+__device__ __forceinline__ int snake_unit(int k, int i, int n) {
+    return k * n + ((k & 1) ? (n - 1 - i) : i);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     gqa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -138,14 +163,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    int b, g;
-    SubTile st[2];
-    fwd_decode_unit(p, blockIdx.x, b, g, st);
-    const int n_max = max(st[0].n_kv, st[1].n_kv);
+    // Persistent CTA: units blockIdx.x, blockIdx.x + gridDim.x, ... (units are ordered
+    // longest first, so this striding spreads the causal work evenly over the SMs).
+    const int cta = blockIdx.x;
+    const int ncta = gridDim.x;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl->q_full), 1);
+        mbar_init(smem_u32(&ctl->q_empty), 1);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(smem_u32(&ctl->full[i]), 1);
             mbar_init(smem_u32(&ctl->empty[i]), 1);
@@ -154,6 +179,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(smem_u32(&ctl->s_full[s]), 1);
             mbar_init(smem_u32(&ctl->p_full[s]), kFwdRows);
             mbar_init(smem_u32(&ctl->o_full[s]), 1);
+            mbar_init(smem_u32(&ctl->o_empty[s]), kFwdRows);
         }
         mbar_init(smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
@@ -173,44 +199,57 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
+    if (warp < 4) setmaxnreg_dec<kFwdCtlRegs>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const int nq = st[1].n_kv > 0 ? 2 : 1;
-            const uint32_t qbar = smem_u32(&ctl->q_full);
-            mbar_arrive_expect_tx(qbar, nq * kTileBytes);
-            for (int s = 0; s < nq; ++s)
-                for (int c = 0; c < L::kChunks; ++c)
-                    tma_load_4d(sQ + s * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64,
-                                st[s].row0, st[s].head, b);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued[kStages];
             for (int i = 0; i < kStages; ++i) issued[i] = 0;
+            uint32_t q_loads = 0;
+            const uint32_t qbar = smem_u32(&ctl->q_full);
             bool ok = true;
-            for (int j = 0; j < n_max && ok; ++j) {
-                for (int t = 0; t < 2; ++t) {
-                    if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag, p.err,
-                                           p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fbar = smem_u32(&ctl->full[stage]);
-                    mbar_arrive_expect_tx(fbar, kTileBytes);
-                    const CUtensorMap* map = t ? &tm_v : &tm_k;
+            for (int k = 0; k * ncta < p.units && ok; ++k) {
+                const int u = snake_unit(k, cta, ncta);
+                if (u >= p.units) continue;
+                int b, g;
+                SubTile st[2];
+                fwd_decode_unit(p, u, b, g, st);
+                const int n_max = max(st[0].n_kv, st[1].n_kv);
+                // the previous unit's Q K^T products must be done before Q is replaced
+                if (q_loads > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->q_empty), (q_loads - 1) & 1u,
+                                                            abort_flag, p.err, p.timeout_ns)))
+                    break;
+                const int nq = st[1].n_kv > 0 ? 2 : 1;
+                mbar_arrive_expect_tx(qbar, nq * kTileBytes);
+                for (int s = 0; s < nq; ++s)
                     for (int c = 0; c < L::kChunks; ++c)
-                        tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
-                                    j * kFwdKeys, g, b);
-                    ++issued[stage];
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
+                        tma_load_4d(sQ + s * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64,
+                                    st[s].row0, st[s].head, b);
+                ++q_loads;
+                for (int j = 0; j < n_max && ok; ++j) {
+                    for (int t = 0; t < 2; ++t) {
+                        if (!(ok = mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
+                                                     p.err, p.timeout_ns)))
+                            break;
+                        const uint32_t fbar = smem_u32(&ctl->full[stage]);
+                        mbar_arrive_expect_tx(fbar, kTileBytes);
+                        const CUtensorMap* map = t ? &tm_v : &tm_k;
+                        for (int c = 0; c < L::kChunks; ++c)
+                            tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
+                                        j * kFwdKeys, g, b);
+                        ++issued[stage];
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
                 }
             }
             if (*abort_flag) {
                 // let every copy this thread started land before the CTA exits
-                mbar_wait_drain(qbar, 0, p.timeout_ns);
+                if (q_loads) mbar_wait_drain(qbar, (q_loads - 1) & 1u, p.timeout_ns);
                 for (int i = 0; i < kStages; ++i)
                     if (issued[i])
                         mbar_wait_drain(smem_u32(&ctl->full[i]), (issued[i] - 1u) & 1u, p.timeout_ns);
@@ -226,7 +265,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t pph[2] = {0u, 0u};
-            bool ok = mbar_wait_bounded(smem_u32(&ctl->q_full), 0, abort_flag, p.err, p.timeout_ns);
+            uint32_t o_uses[2] = {0u, 0u};  // units whose O_s epilogue must drain first
+            uint32_t q_uses = 0;
+            bool ok = true;
 
             auto acquire = [&](int& slot) -> bool {
                 slot = stage;
@@ -263,41 +304,64 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             };
 
-            int kslot = 0;
-            if (ok && n_max > 0) ok = acquire(kslot);
-            if (ok && n_max > 0) {
+            for (int k = 0; k * ncta < p.units && ok; ++k) {
+                const int u = snake_unit(k, cta, ncta);
+                if (u >= p.units) continue;
+                int b, g;
+                SubTile st[2];
+                fwd_decode_unit(p, u, b, g, st);
+                const int n_max = max(st[0].n_kv, st[1].n_kv);
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->q_full), q_uses & 1u, abort_flag, p.err,
+                                             p.timeout_ns)))
+                    break;
+                ++q_uses;
+                int kslot;
+                if (!(ok = acquire(kslot))) break;
                 for (int s = 0; s < 2; ++s)
                     if (st[s].n_kv > 0) {
                         issue_qk(s, kslot);
                         tc_commit(smem_u32(&ctl->s_full[s]));
                     }
                 tc_commit(smem_u32(&ctl->empty[kslot]));
-            }
-            for (int j = 0; j < n_max && ok; ++j) {
-                int vslot;
-                if (!(ok = acquire(vslot))) break;
-                const bool next = j + 1 < n_max;
-                int knext = -1;
-                for (int s = 0; s < 2 && ok; ++s) {
-                    if (j < st[s].n_kv) {
-                        if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full[s]), pph[s], abort_flag,
-                                                     p.err, p.timeout_ns)))
-                            break;
-                        pph[s] ^= 1u;
-                        tc_fence_after_sync();
-                        issue_pv(s, vslot, j > 0);
-                        if (j == st[s].n_kv - 1) tc_commit(smem_u32(&ctl->o_full[s]));
-                    }
-                    if (s == 1) tc_commit(smem_u32(&ctl->empty[vslot]));
-                    if (next) {
-                        if (knext < 0 && !(ok = acquire(knext))) break;
-                        if (j + 1 < st[s].n_kv) {
-                            issue_qk(s, knext);
-                            tc_commit(smem_u32(&ctl->s_full[s]));
+                if (n_max == 1) tc_commit(smem_u32(&ctl->q_empty));
+                for (int j = 0; j < n_max && ok; ++j) {
+                    int vslot;
+                    if (!(ok = acquire(vslot))) break;
+                    const bool next = j + 1 < n_max;
+                    int knext = -1;
+                    for (int s = 0; s < 2 && ok; ++s) {
+                        if (j < st[s].n_kv) {
+                            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full[s]), pph[s], abort_flag,
+                                                         p.err, p.timeout_ns)))
+                                break;
+                            pph[s] ^= 1u;
+                            if (j == 0 && o_uses[s] > 0) {
+                                // the previous unit's epilogue must have read O_s
+                                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->o_empty[s]), (o_uses[s] - 1) & 1u,
+                                                             abort_flag, p.err, p.timeout_ns)))
+                                    break;
+                            }
+                            tc_fence_after_sync();
+                            issue_pv(s, vslot, j > 0);
+                            if (j == st[s].n_kv - 1) {
+                                tc_commit(smem_u32(&ctl->o_full[s]));
+                                ++o_uses[s];
+                            }
+                        }
+                        if (s == 1) tc_commit(smem_u32(&ctl->empty[vslot]));
+                        if (next) {
+                            if (knext < 0 && !(ok = acquire(knext))) break;
+                            if (j + 1 < st[s].n_kv) {
+                                issue_qk(s, knext);
+                                tc_commit(smem_u32(&ctl->s_full[s]));
+                            }
                         }
                     }
+                    if (ok && next) {
+                        tc_commit(smem_u32(&ctl->empty[knext]));
+                        if (j + 2 == n_max) tc_commit(smem_u32(&ctl->q_empty));  // last Q K^T issued
+                    }
                 }
-                if (ok && next) tc_commit(smem_u32(&ctl->empty[knext]));
             }
             if (*abort_flag) {
                 // wait for the MMAs already issued before TMEM is released
@@ -307,21 +371,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax warpgroups
+        setmaxnreg_inc<kFwdSoftmaxRegs>();
         const int s = (warp - 4) >> 2;
         const int quad = warp & 3;         // TMEM lane quadrant this warp may access
         const int r = quad * 32 + lane;    // row within the sub-tile
-        const SubTile me = st[s];
-        if (me.n_kv > 0) {
-            const int off = p.Tk - p.Tq;
+        const uint32_t lane_sel = (uint32_t)(quad * 32) << 16;
+        const uint32_t tS = tmem + lane_sel + (uint32_t)(s * 128);
+        const uint32_t tO = tmem + lane_sel + 256u + (uint32_t)(s * D);
+        const float sl2 = p.scale_log2;
+        const int off = p.Tk - p.Tq;
+        uint32_t sph = 0, oph = 0;
+        bool ok = true;
+        for (int k = 0; k * ncta < p.units && ok; ++k) {
+            const int u = snake_unit(k, cta, ncta);
+            if (u >= p.units) continue;
+            int b, g;
+            SubTile st[2];
+            fwd_decode_unit(p, u, b, g, st);
+            const SubTile me = st[s];
+            if (me.n_kv == 0) continue;
             const int pos = off + me.row0 + r;  // absolute position of this query row
-            const uint32_t lane_sel = (uint32_t)(quad * 32) << 16;
-            const uint32_t tS = tmem + lane_sel + (uint32_t)(s * 128);
-            const uint32_t tO = tmem + lane_sel + 256u + (uint32_t)(s * D);
-            const float sl2 = p.scale_log2;
             float m = -INFINITY;  // running max of scaled scores (log2 units)
             float l = 0.f;        // running sum of exp2(score - m)
-            uint32_t sph = 0;
-            bool ok = true;
             for (int j = 0; j < me.n_kv; ++j) {
                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full[s]), sph, abort_flag, p.err,
                                              p.timeout_ns)))
@@ -332,8 +403,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
                 tc_wait_ld();
-                float tmax = -INFINITY;
-                if (j >= me.masked_from) {
+                const bool diag = j >= me.masked_from;
+                if (diag) {
                     const int lim = pos - j * kFwdKeys;  // columns > lim are in the future
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
@@ -342,10 +413,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             if (c * 32 + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
                         }
                 }
+                // row max: eight independent chains of 3-input max, then a small tree
+                float mx[8];
+#pragma unroll
+                for (int qd = 0; qd < 8; ++qd) mx[qd] = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(sr[c][e]));
+                    for (int qd = 0; qd < 8; ++qd) {
+                        mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd]), __uint_as_float(sr[c][4 * qd + 1]));
+                        mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd + 2]), __uint_as_float(sr[c][4 * qd + 3]));
+                    }
+                const float tmax = fmaxf(max3f(mx[0], mx[1], mx[2]),
+                                         max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
                 const float m_new = fmaxf(m, tmax * sl2);
                 const bool refresh = m_new > m + kRescaleThreshold;
                 float alpha = 1.f;
@@ -369,49 +449,85 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     }
                 }
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t negm2 = f2_pack(neg_m, neg_m);
+                uint64_t lacc[4] = {0ull, 0ull, 0ull, 0ull};
+                // p = 2^(s * scale * log2(e) - m), two columns per packed instruction; on
+                // tiles without masked columns every kPolyEvery-th pair goes through the
+                // FMA-pipe polynomial so the MUFU is not the only exp2 unit.
+                auto exp_pair = [&](uint64_t x, bool poly) -> uint64_t {
+                    if (poly) return exp2_poly_x2(x);
+                    float x0, x1;
+                    f2_unpack(x, x0, x1);
+                    return f2_pack(ex2_approx(x0), ex2_approx(x1));
+                };
+                auto softmax_chunks = [&](auto poly_tag) {
+                    constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, neg_m));
-                        l += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t x = f2_fma(
+                                f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                                sl2x2, negm2);
+                            const bool use_poly =
+                                kPoly && kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+                            const uint64_t pp = exp_pair(x, use_poly);
+                            lacc[e & 3] = f2_add(lacc[e & 3], pp);
+                            float p0, p1;
+                            f2_unpack(pp, p0, p1);
+                            pk[e] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(tS + c * 16, pk);
                     }
-                    tmem_st16(tS + c * 16, pk);
+                };
+                if (diag)
+                    softmax_chunks(std::false_type{});
+                else
+                    softmax_chunks(std::true_type{});
+
+                {
+                    const uint64_t s01 = f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3]));
+                    float a0, a1;
+                    f2_unpack(s01, a0, a1);
+                    l += a0 + a1;
                 }
                 tc_wait_st();
                 tc_fence_before_sync();
                 mbar_arrive(smem_u32(&ctl->p_full[s]));
             }
-            if (ok && mbar_wait_bounded(smem_u32(&ctl->o_full[s]), 0, abort_flag, p.err, p.timeout_ns)) {
-                tc_fence_after_sync();
-                const int row = me.row0 + r;
-                const float inv_l = 1.f / l;
-                __nv_bfloat16* out =
-                    p.o + (((size_t)b * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
+            if (!ok || !(ok = mbar_wait_bounded(smem_u32(&ctl->o_full[s]), oph, abort_flag, p.err,
+                                                p.timeout_ns)))
+                break;
+            oph ^= 1u;
+            tc_fence_after_sync();
+            const int row = me.row0 + r;
+            const float inv_l = 1.f / l;
+            __nv_bfloat16* out = p.o + (((size_t)b * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO + c * 32, orr);
-                    tc_wait_ld();
-                    uint4 v4[4];
-                    uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t orr[32];
+                tmem_ld32(tO + c * 32, orr);
+                tc_wait_ld();
+                uint4 v4[4];
+                uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pw[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
-                                            __uint_as_float(orr[2 * e + 1]) * inv_l);
-                    if (row < p.Tq) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+                for (int e = 0; e < 16; ++e)
+                    pw[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
+                                        __uint_as_float(orr[2 * e + 1]) * inv_l);
+                if (row < p.Tq) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = v4[e];
-                    }
+                    for (int e = 0; e < 4; ++e) dst[e] = v4[e];
                 }
-                if (p.lse != nullptr && row < p.Tq)
-                    p.lse[((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row] =
-                        (m + __log2f(l)) * 0.69314718055994530942f;
             }
+            // O_s has been read: the next unit's first P V may overwrite it
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&ctl->o_empty[s]));
+            if (p.lse != nullptr && row < p.Tq)
+                p.lse[((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row] =
+                    (m + __log2f(l)) * 0.69314718055994530942f;
         }
     }
 

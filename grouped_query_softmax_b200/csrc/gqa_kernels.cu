@@ -3,6 +3,8 @@
 // relocatable device code.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "gqa_internal.h"
@@ -44,11 +46,24 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     p.timeout_ns = kWaitTimeoutNs;
     if (!p.err) return cudaErrorUnknown;
     if (units <= 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const int smem = FwdSmem<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    p.units = (int)units;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    gqa_fwd_sm100_kernel<D><<<(unsigned)units, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int smem = FwdSmem<D>::kBytes;
+    e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    // The in-kernel register split (setmaxnreg) needs exactly the launch allocation it
+    // was sized for; never launch a build where that does not hold.
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, gqa_fwd_sm100_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
+    // persistent: one CTA per SM (shared memory and TMEM allow exactly one)
+    const unsigned grid = (unsigned)std::min<long long>(units, sms > 0 ? sms : 1);
+    gqa_fwd_sm100_kernel<D><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
     return cudaGetLastError();
 }
 

@@ -204,6 +204,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// Per-warpgroup register budget changes; every thread of the warpgroup executes them.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor"): start address,
 // leading/stride byte offsets (all >> 4), version 1 at bits 46-47, swizzle mode at
@@ -238,6 +248,60 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic): one instruction for two lanes of work.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU: Cody-Waite style range
+// reduction x = n + f with n = rint(x) (obtained by adding 1.5 * 2^23, which leaves n
+// in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients were fitted for this library as the minimax relative-error fit on
+// [-1/2, 1/2] (max relative error 7.5e-5 after fp32 evaluation); 2^n is applied by
+// adding n to the exponent field. Inputs are clamped to >= -125 so the result stays
+// a normal number; callers only use it where no input is -inf.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+    const uint64_t t = f2_add(x, magic);
+    const uint64_t f = f2_sub(x, f2_sub(t, magic));
+    uint64_t p = f2_fma(f2_pack(0.05517221987247467f, 0.05517221987247467f), f,
+                        f2_pack(0.24261115491390228f, 0.24261115491390228f));
+    p = f2_fma(p, f, f2_pack(0.6932608485221863f, 0.6932608485221863f));
+    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    const uint32_t tl = (uint32_t)t, th = (uint32_t)(t >> 32);
+    const uint32_t pl = (uint32_t)p + (tl << 23), ph = (uint32_t)(p >> 32) + (th << 23);
+    return ((uint64_t)ph << 32) | pl;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
