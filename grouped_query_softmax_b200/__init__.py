@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "GqaError", "gqa_attn_fwd", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
-    "gqa_attn_decode_num_splits", "gqa_status_string", "gqa_get_device_error",
+    "gqa_attn_decode_num_splits", "gqa_attn_decode_static", "gqa_status_string", "gqa_get_device_error",
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
@@ -53,6 +53,9 @@ _lib.gqa_attn_decode_num_splits.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.gqa_attn_decode.restype = _i32
 _lib.gqa_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                  _ll, _ll, _ll, _ll, _f32, _i32, _vp, _sz, _vp]
+_lib.gqa_attn_decode_static.restype = _i32
+_lib.gqa_attn_decode_static.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                        _ll, _ll, _ll, _ll, _f32, _i32, _vp]
 _lib.gqa_status_string.restype = ctypes.c_char_p
 _lib.gqa_status_string.argtypes = [_i32]
 _lib.gqa_get_device_error.restype = _i32
@@ -93,6 +96,14 @@ def gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb,
     """C ``gqa_attn_decode``; pointers are integers (device addresses). Returns the status."""
     return _lib.gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
                                 float(softmax_scale), num_splits, workspace, workspace_bytes, stream)
+
+
+def gqa_attn_decode_static(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                           softmax_scale=0.0, num_splits=0, stream=None) -> int:
+    """C ``gqa_attn_decode_static``: decode with the library's fixed 16 MiB device scratch
+    instead of a caller workspace, for callers that cannot allocate device memory."""
+    return _lib.gqa_attn_decode_static(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb,
+                                       v_sh, float(softmax_scale), num_splits, stream)
 
 
 def gqa_status_string(status: int) -> str:

@@ -103,6 +103,29 @@ GQA_API gqa_status gqa_attn_decode(const void* q, const void* k_cache, const voi
                            float softmax_scale, int num_splits,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Decode for callers that cannot allocate device memory at call time (for example a
+ * plugin running inside an engine that owns all device memory, or a decode loop that
+ * forbids cudaMalloc because it may synchronise the device). The pages have no
+ * counterpart: this is a library convenience around gqa_attn_decode.
+ *
+ * Same arguments and results as gqa_attn_decode without the workspace. The split-KV
+ * partials live in a 16 MiB scratch array compiled into the library: one per device
+ * that loads the library, held until the process exits. A call whose partials need
+ * more (gqa_attn_decode_workspace_bytes(...) > 16 MiB) returns GQA_ERR_WORKSPACE and
+ * launches nothing; num_splits = 1 needs no scratch. Allocates nothing.
+ * The first call on each device does a one-time set-up (it looks up the scratch's
+ * device address); make that first call before any stream capture. All calls on a
+ * device share the scratch and it keeps the last call's contents (nothing needs
+ * clearing: every partial is written before it is read); calls whose kernels can
+ * overlap on the GPU race on it.
+ */
+GQA_API gqa_status gqa_attn_decode_static(const void* q, const void* k_cache, const void* v_cache,
+                                          void* o, int B, int Hq, int Hkv, int Tk, int D,
+                                          long long k_sb, long long k_sh, long long v_sb,
+                                          long long v_sh, float softmax_scale, int num_splits,
+                                          void* stream);
+
 /* The split count gqa_attn_decode will use for these arguments (num_splits 0 = auto). */
 GQA_API int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits);
 
