@@ -283,18 +283,23 @@ def oracle_sample(w, budget_s: float, threads: int, q=None, k=None, v=None):
         q, k, v = w.make()
     rng = np.random.default_rng(0)
     total = w.B * w.Hq * w.Tq
-    probe = rng.integers(0, total, size=min(total, max(threads, 16)))
+    # calibrate the parallel rate on a probe of several rows per thread
+    probe = rng.integers(0, total, size=min(total, 8 * threads))
     t = time.perf_counter()
     oracle.attention_rows(q, k, v, probe, threads=threads)
     dt = max(time.perf_counter() - t, 1e-6)
     rate = row_flops(w, probe) / dt
-    mean_row = row_flops(w, np.arange(total)) / total if total <= 1 << 22 else 4.0 * w.D * (
-        w.Tk - w.Tq + w.Tq / 2)
-    n = int(min(total, max(threads, budget_s * rate / mean_row)))
-    rows = np.sort(rng.choice(total, size=n, replace=False)) if n < total else np.arange(total)
-    t = time.perf_counter()
-    oracle.attention_rows(q, k, v, rows, threads=threads)
-    dt = time.perf_counter() - t
+    mean_row = 4.0 * w.D * (w.Tk - w.Tq + (w.Tq + 1) / 2)
+    n = int(min(total, max(8 * threads, budget_s * rate / mean_row)))
+    for _ in range(3):
+        rows = np.sort(rng.choice(total, size=n, replace=False)) if n < total else np.arange(total)
+        t = time.perf_counter()
+        oracle.attention_rows(q, k, v, rows, threads=threads)
+        dt = time.perf_counter() - t
+        if dt >= 0.5 * budget_s or n >= total:
+            break
+        # the probe under-estimated the parallel rate: resize from the measured run
+        n = int(min(total, n * budget_s / max(dt, 1e-3)))
     return row_flops(w, rows), dt, rows
 
 
@@ -318,6 +323,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the main workload's batch size (for profiling a smaller case)")
     return ap.parse_args(argv)
 
 
@@ -395,6 +402,9 @@ def main(argv=None):
 
     peaks, peak_src = load_peaks()
     w = gi.WORKLOADS[args.workload]
+    if args.batch > 0:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name} (batch {args.batch})")
     gpu_id = None
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:

@@ -1,0 +1,49 @@
+"""The bench's multi-rank plumbing on CPU: two gloo ranks, each with its own
+independent problem (weak scaling, no data-path collective); the timed value is the
+max over ranks and the reported throughput counts every rank's work."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    import bench
+    r, w, local = bench.dist_env()
+    assert (r, w, local) == (rank, world, rank)
+    bench.barrier(w)
+    worst = bench.max_over_ranks(10.0 + rank, w)          # rank 1 is the slower one
+    wl = bench.gi.WORKLOADS["gqa_prefill"]
+    one = bench.throughput(wl, worst, 1)
+    agg = bench.throughput(wl, worst, w)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, worst, one, agg))
+
+
+def test_two_gloo_ranks_take_the_max_time_and_aggregate_work():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, worst, one, agg in res:
+        assert worst == 11.0
+        assert agg == pytest.approx(2 * one)
