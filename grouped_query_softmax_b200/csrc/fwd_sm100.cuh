@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kFwdRows, D, 0, 1);
             const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
+            // descriptors advance by constants (their start-address field is in 16-byte units)
+            const uint64_t desc_q[2] = {umma_desc_sw128(sQ, 16, 1024), umma_desc_sw128(sQ + kTileBytes, 16, 1024)};
             int stage = 0;
             uint32_t phase = 0;
             uint32_t pph[2] = {0u, 0u};
@@ -284,24 +286,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // S_s = Q_s K^T: M=128 rows, N=128 keys, K=D in steps of 16 (32 bytes of a
             // 128-byte swizzled row; the next 64 columns live in the next chunk).
             auto issue_qk = [&](int s, int kslot) {
+                const uint64_t a0 = desc_q[s];
+                const uint64_t b0 = umma_desc_sw128(sRing + kslot * kTileBytes, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-                    const uint64_t a = umma_desc_sw128(sQ + s * kTileBytes + koff, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(sRing + kslot * kTileBytes + koff, 16, 1024);
-                    tc_mma_ss(tS[s], a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t koff = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tS[s], a0 + koff, b0 + koff, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
             // O_s += P_s V: M=128 rows, N=D, K=128 keys in steps of 16. P (bf16, two per
             // column) sits in the first 64 columns of S_s; V is N-contiguous (d), with
             // the 64-column chunks LBO apart and 8-key groups 1024 bytes apart.
             auto issue_pv = [&](int s, int vslot, bool accumulate) {
+                const uint64_t b0 = umma_desc_sw128(sRing + vslot * kTileBytes, kChunkBytes, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kFwdKeys / 16; ++kk) {
-                    const uint64_t bd =
-                        umma_desc_sw128(sRing + vslot * kTileBytes + kk * 2048, kChunkBytes, 1024);
-                    tc_mma_ts(tO[s], tS[s] + kk * 8, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kFwdKeys / 16; ++kk)
+                    tc_mma_ts(tO[s], tS[s] + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                              (accumulate || kk > 0) ? 1u : 0u);
             };
 
             for (int k = 0; k * ncta < p.units && ok; ++k) {
@@ -400,10 +401,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 sph ^= 1u;
                 tc_fence_after_sync();
                 uint32_t sr[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                tmem_ld32(tS + 0, sr[0]);
+                tmem_ld32(tS + 32, sr[1]);
                 tc_wait_ld();
+                reg_fence32(sr[0]);
+                reg_fence32(sr[1]);
+                tmem_ld32(tS + 64, sr[2]);
+                tmem_ld32(tS + 96, sr[3]);
                 const bool diag = j >= me.masked_from;
+                // row max: eight independent chains of 3-input max, then a small tree; the
+                // first 64 columns are reduced while the last 64 are still loading
+                float mx[8];
+#pragma unroll
+                for (int qd = 0; qd < 8; ++qd) mx[qd] = -INFINITY;
+                if (!diag) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+#pragma unroll
+                        for (int qd = 0; qd < 8; ++qd) {
+                            mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd]), __uint_as_float(sr[c][4 * qd + 1]));
+                            mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd + 2]), __uint_as_float(sr[c][4 * qd + 3]));
+                        }
+                }
+                tc_wait_ld();
+                reg_fence32(sr[2]);
+                reg_fence32(sr[3]);
                 if (diag) {
                     const int lim = pos - j * kFwdKeys;  // columns > lim are in the future
 #pragma unroll
@@ -413,17 +435,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             if (c * 32 + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
                         }
                 }
-                // row max: eight independent chains of 3-input max, then a small tree
-                float mx[8];
 #pragma unroll
-                for (int qd = 0; qd < 8; ++qd) mx[qd] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 4; ++c) {
+                    if (!diag && c < 2) continue;  // already reduced
 #pragma unroll
                     for (int qd = 0; qd < 8; ++qd) {
                         mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd]), __uint_as_float(sr[c][4 * qd + 1]));
                         mx[qd] = max3f(mx[qd], __uint_as_float(sr[c][4 * qd + 2]), __uint_as_float(sr[c][4 * qd + 3]));
                     }
+                }
                 const float tmax = fmaxf(max3f(mx[0], mx[1], mx[2]),
                                          max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
                 const float m_new = fmaxf(m, tmax * sl2);
@@ -442,6 +462,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         uint32_t orr[32];
                         tmem_ld32(tO + c * 32, orr);
                         tc_wait_ld();
+                        reg_fence32(orr);
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
@@ -510,6 +531,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 uint32_t orr[32];
                 tmem_ld32(tO + c * 32, orr);
                 tc_wait_ld();
+                reg_fence32(orr);
                 uint4 v4[4];
                 uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
 #pragma unroll
