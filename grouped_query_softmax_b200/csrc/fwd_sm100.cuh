@@ -329,7 +329,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     int vslot;
                     if (!(ok = acquire(vslot))) break;
                     const bool next = j + 1 < n_max;
+                    // take the next K slot now, so each Q K^T follows its P V on the tensor
+                    // pipe with no gap
                     int knext = -1;
+                    if (next && !(ok = acquire(knext))) break;
                     for (int s = 0; s < 2 && ok; ++s) {
                         if (j < st[s].n_kv) {
                             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full[s]), pph[s], abort_flag,
@@ -351,7 +354,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         }
                         if (s == 1) tc_commit(smem_u32(&ctl->empty[vslot]));
                         if (next) {
-                            if (knext < 0 && !(ok = acquire(knext))) break;
                             if (j + 1 < st[s].n_kv) {
                                 issue_qk(s, knext);
                                 tc_commit(smem_u32(&ctl->s_full[s]));
@@ -448,12 +450,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                          max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
                 const float m_new = fmaxf(m, tmax * sl2);
                 const bool refresh = m_new > m + kRescaleThreshold;
-                float alpha = 1.f;
-                if (refresh) {
-                    alpha = ex2_approx(m - m_new);
-                    l *= alpha;
-                    m = m_new;
-                }
+                const float alpha = refresh ? ex2_approx(m - m_new) : 1.f;
+                l *= alpha;
+                m = refresh ? m_new : m;
                 if (j > 0 && __any_sync(0xffffffffu, refresh)) {
                     // O_s has absorbed all earlier P V products (their completion is
                     // ordered before S_j's commit); rescale this row in place.
