@@ -41,6 +41,10 @@ def _bind(lib):
     lib.gqa_oracle_rows.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                     ll, ll, ll, ll, ll, ll, ctypes.c_double,
                                     vp, ll, vp, vp, i32]
+    lib.gqa_oracle_rows_window.restype = i32
+    lib.gqa_oracle_rows_window.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                           ll, ll, ll, ll, ll, ll, ctypes.c_double, i32,
+                                           vp, ll, vp, vp, i32]
     return lib
 
 
@@ -68,13 +72,14 @@ def _plane_strides(arr: np.ndarray, name: str):
 
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows, Tk: int | None = None,
                    scale: float | None = None, threads: int | None = None, with_lse: bool = False,
-                   lib=None):
+                   lib=None, window: int = 0):
     """fp64 output rows of causal GQA attention.
 
     q: uint16 [B, H_q, T_q, D]; k, v: uint16 [B, H_kv, T_cap, D] (rows packed,
     batch/head strides free; only the first ``Tk`` positions are read, default
-    T_cap). ``rows`` are flat ids (b*H_q + a)*T_q + i. Returns a float64
-    [len(rows), D] array (and the natural-log LSE per row if ``with_lse``).
+    T_cap). ``rows`` are flat ids (b*H_q + a)*T_q + i. ``window`` > 0 restricts each
+    query to its ``window`` most recent positions. Returns a float64 [len(rows), D]
+    array (and the natural-log LSE per row if ``with_lse``).
     """
     B, Hq, Tq, D = q.shape
     Bk, Hkv, Tcap, Dk = k.shape
@@ -87,9 +92,9 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows, Tk: int | 
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
     out = np.empty((rows.size, D), dtype=np.float64)
     lse = np.empty(rows.size, dtype=np.float64) if with_lse else None
-    rc = (lib or _load()).gqa_oracle_rows(
+    rc = (lib or _load()).gqa_oracle_rows_window(
         q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Hq, Hkv, Tq, Tk, D,
-        q_sb, q_sh, k_sb, k_sh, v_sb, v_sh, float(scale) if scale else 0.0,
+        q_sb, q_sh, k_sb, k_sh, v_sb, v_sh, float(scale) if scale else 0.0, int(window),
         rows.ctypes.data, rows.size, out.ctypes.data, lse.ctypes.data if with_lse else None,
         int(threads or default_threads()))
     if rc == 1:
@@ -101,11 +106,11 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows, Tk: int | 
 
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, Tk: int | None = None,
               scale: float | None = None, threads: int | None = None, with_lse: bool = False,
-              lib=None):
+              lib=None, window: int = 0):
     """All output rows, shaped [B, H_q, T_q, D] (float64)."""
     B, Hq, Tq, D = q.shape
     res = attention_rows(q, k, v, np.arange(B * Hq * Tq), Tk=Tk, scale=scale, threads=threads,
-                         with_lse=with_lse, lib=lib)
+                         with_lse=with_lse, lib=lib, window=window)
     if with_lse:
         return res[0].reshape(B, Hq, Tq, D), res[1].reshape(B, Hq, Tq)
     return res.reshape(B, Hq, Tq, D)

@@ -21,6 +21,11 @@
  *        section Mask 与增量位置; "A Visual Guide to Attention", section
  *        "Which positions are visible?".
  *   Scale 1/sqrt(D) with D the head dimension (the ABI allows an override).
+ *   Optional sliding window w > 0: the query at position p sees only its w most
+ *   recent positions, keys j with p - w < j <= p (itself included)
+ *     -- "A Visual Guide to Attention", section "Which positions are visible?"
+ *        (sliding-window attention keeps the most recent w positions directly
+ *        visible); w <= 0 means plain causal attention.
  *
  * Precision: every input is a bf16 value, widened exactly to double; all
  * arithmetic is double; nothing is rounded to a lower precision. Subtracting
@@ -51,6 +56,7 @@ typedef struct {
     int B, Hq, Hkv, Tq, Tk, D;
     long long q_sb, q_sh, k_sb, k_sh, v_sb, v_sh;
     double scale;
+    int window; /* <= 0: causal only */
     const long long* rows;
     long long n_rows;
     double* out;
@@ -75,9 +81,12 @@ static void oracle_row(const oracle_job* J, long long row, double* s, double* qd
 
     for (int d = 0; d < D; ++d) qd[d] = bf16_to_double(qrow[d]);
 
-    /* scores s_j = scale * <q_i, k_j> for visible keys j = 0..pos */
+    /* first visible key: 0 for causal attention, pos - w + 1 inside a window of w */
+    const long long first = (J->window > 0 && pos - J->window + 1 > 0) ? pos - J->window + 1 : 0;
+
+    /* scores s_j = scale * <q_i, k_j> for visible keys j = first..pos */
     double m = -INFINITY;
-    for (long long j = 0; j <= pos; ++j) {
+    for (long long j = first; j <= pos; ++j) {
         const uint16_t* krow = kplane + j * D;
         double acc = 0.0;
         for (int d = 0; d < D; ++d) acc += qd[d] * bf16_to_double(krow[d]);
@@ -86,13 +95,13 @@ static void oracle_row(const oracle_job* J, long long row, double* s, double* qd
     }
     /* softmax weights and normaliser */
     double l = 0.0;
-    for (long long j = 0; j <= pos; ++j) {
+    for (long long j = first; j <= pos; ++j) {
         s[j] = exp(s[j] - m);
         l += s[j];
     }
     /* weighted sum of value rows */
     for (int d = 0; d < D; ++d) o[d] = 0.0;
-    for (long long j = 0; j <= pos; ++j) {
+    for (long long j = first; j <= pos; ++j) {
         const uint16_t* vrow = vplane + j * D;
         const double w = s[j];
         for (int d = 0; d < D; ++d) o[d] += w * bf16_to_double(vrow[d]);
@@ -129,11 +138,11 @@ static void* oracle_worker(void* arg) {
  * scale <= 0 selects 1/sqrt(D). n_threads <= 0 selects one thread.
  * Returns 0 on success, 1 on invalid arguments, 2 on allocation failure.
  */
-int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
-                    int Hkv, int Tq, int Tk, int D, long long q_sb, long long q_sh,
-                    long long k_sb, long long k_sh, long long v_sb, long long v_sh, double scale,
-                    const long long* rows, long long n_rows, double* out, double* lse,
-                    int n_threads) {
+int gqa_oracle_rows_window(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                           int Hkv, int Tq, int Tk, int D, long long q_sb, long long q_sh,
+                           long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                           double scale, int window, const long long* rows, long long n_rows,
+                           double* out, double* lse, int n_threads) {
     if (!q || !k || !v || !out || (!rows && n_rows > 0)) return 1;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || D <= 0) return 1;
     if (Hq % Hkv != 0 || Tq > Tk) return 1; /* the pages' asserted preconditions */
@@ -146,6 +155,7 @@ int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Tq = Tq; J.Tk = Tk; J.D = D;
     J.q_sb = q_sb; J.q_sh = q_sh; J.k_sb = k_sb; J.k_sh = k_sh; J.v_sb = v_sb; J.v_sh = v_sh;
     J.scale = scale > 0.0 ? scale : 1.0 / sqrt((double)D);
+    J.window = window;
     J.rows = rows; J.n_rows = n_rows; J.out = out; J.lse = lse; J.next = 0;
 
     if (n_threads <= 1) return oracle_worker(&J) ? 2 : 0;
@@ -165,4 +175,14 @@ int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
     for (int t = 0; t < n_threads; ++t) any |= started[t];
     if (!any) rc = oracle_worker(&J) ? 2 : 0;
     return rc;
+}
+
+/* Plain causal attention (no window). */
+int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                    int Hkv, int Tq, int Tk, int D, long long q_sb, long long q_sh,
+                    long long k_sb, long long k_sh, long long v_sb, long long v_sh, double scale,
+                    const long long* rows, long long n_rows, double* out, double* lse,
+                    int n_threads) {
+    return gqa_oracle_rows_window(q, k, v, B, Hq, Hkv, Tq, Tk, D, q_sb, q_sh, k_sb, k_sh, v_sb, v_sh,
+                                  scale, 0, rows, n_rows, out, lse, n_threads);
 }

@@ -11,8 +11,11 @@ matrices, so a slip in the oracle's indices shows up as a mismatch here.
 import numpy as np
 
 
-def brute_force_attention(qf: np.ndarray, kf: np.ndarray, vf: np.ndarray, scale=None):
-    """qf [B,Hq,Tq,D], kf/vf [B,Hkv,Tk,D], float64 values. Returns [B,Hq,Tq,D]."""
+def brute_force_attention(qf: np.ndarray, kf: np.ndarray, vf: np.ndarray, scale=None, window=0):
+    """qf [B,Hq,Tq,D], kf/vf [B,Hkv,Tk,D], float64 values. Returns [B,Hq,Tq,D].
+
+    window > 0 adds the sliding-window mask: keys more than window-1 positions
+    before the query are hidden too."""
     B, Hq, Tq, D = qf.shape
     Hkv, Tk = kf.shape[1], kf.shape[2]
     assert Hq % Hkv == 0 and Tq <= Tk
@@ -23,7 +26,10 @@ def brute_force_attention(qf: np.ndarray, kf: np.ndarray, vf: np.ndarray, scale=
     scores = np.matmul(qf, np.swapaxes(k_exp, -1, -2)) * scale  # [B,Hq,Tq,Tk]
     query_pos = np.arange(Tk - Tq, Tk)[:, None]
     key_pos = np.arange(Tk)[None, :]
-    mask = np.where(key_pos > query_pos, -np.inf, 0.0)  # [Tq,Tk]
+    hidden = key_pos > query_pos
+    if window > 0:
+        hidden = hidden | (key_pos <= query_pos - window)
+    mask = np.where(hidden, -np.inf, 0.0)  # [Tq,Tk]
     scores = scores + mask
     scores = scores - scores.max(axis=-1, keepdims=True)
     w = np.exp(scores)

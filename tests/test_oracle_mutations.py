@@ -29,6 +29,11 @@ MUTATIONS = [
     ("batch stride of K dropped", "J->k + b * J->k_sb + g * J->k_sh", "J->k + g * J->k_sh"),
     ("LSE without log", "*lse_out = m + log(l);", "*lse_out = m + l;"),
     ("query and key swapped in the group", "a / group;", "a / J->Hkv;"),
+    ("window one key too wide", "pos - J->window + 1 > 0) ? pos - J->window + 1 : 0;",
+     "pos - J->window > 0) ? pos - J->window : 0;"),
+    ("window one key too narrow", "pos - J->window + 1 > 0) ? pos - J->window + 1 : 0;",
+     "pos - J->window + 2 > 0) ? pos - J->window + 2 : 0;"),
+    ("window ignored", "(J->window > 0 && pos", "(0 && pos"),
 ]
 
 PIN_TESTS = [
@@ -43,6 +48,9 @@ PIN_TESTS = [
     (pins.test_gqa_equals_mha_on_repeated_planes, {}),
     (pins.test_affine_in_values, {}),
     (pins.test_row_subset_matches_full_and_strided_cache, {}),
+    (pins.test_window_of_one_returns_the_own_value_row, {}),
+    (pins.test_window_zero_query_gives_window_mean, {}),
+    (pins.test_window_matches_brute_force_matrix_form, {"shape": (2, 4, 2, 9, 9, 8), "w": 3}),
 ]
 
 

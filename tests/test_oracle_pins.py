@@ -209,3 +209,56 @@ def test_rejects_what_the_pages_assert_against():
 def test_threads_do_not_change_results():
     q, k, v = rand_qkv(2, 4, 2, 33, 40, 16, seed=4)
     np.testing.assert_array_equal(att(q, k, v, threads=1), att(q, k, v, threads=8))
+
+
+# ---------------------------------------------------------------- sliding window
+def test_window_of_one_returns_the_own_value_row():
+    """w = 1: each query sees only its own position, so o = v[pos] and LSE = its own score."""
+    B, Hq, Hkv, Tq, Tk, D = 1, 4, 2, 6, 9, 8
+    q, k, v = rand_qkv(B, Hq, Hkv, Tq, Tk, D, seed=31)
+    out, lse = att(q, k, v, window=1, with_lse=True)
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    for a in range(Hq):
+        g = a // (Hq // Hkv)
+        for i in range(Tq):
+            pos = Tk - Tq + i
+            np.testing.assert_array_equal(out[0, a, i], vf[0, g, pos])
+            assert abs(lse[0, a, i] - qf[0, a, i] @ kf[0, g, pos] / math.sqrt(D)) < 1e-12
+
+
+def test_window_zero_query_gives_window_mean():
+    """q = 0 inside a window of w: o_i is the mean of v over positions max(0, pos-w+1)..pos."""
+    B, Hq, Hkv, Tq, Tk, D, w = 1, 2, 1, 7, 13, 8, 4
+    _, k, v = rand_qkv(B, Hq, Hkv, Tq, Tk, D, seed=33)
+    q = bits(np.zeros((B, Hq, Tq, D)))
+    out, lse = att(q, k, v, window=w, with_lse=True)
+    vf = f64(v)
+    for i in range(Tq):
+        pos = Tk - Tq + i
+        lo = max(0, pos - w + 1)
+        np.testing.assert_allclose(out[0, 0, i], vf[0, 0, lo:pos + 1].mean(axis=0), rtol=0, atol=1e-14)
+        assert abs(lse[0, 0, i] - math.log(pos + 1 - lo)) < 1e-14
+
+
+@pytest.mark.parametrize("shape,w", [((2, 4, 2, 9, 9, 8), 3), ((1, 4, 1, 5, 12, 4), 5), ((1, 3, 3, 8, 8, 16), 1),
+                                     ((2, 2, 1, 1, 10, 8), 4)])
+def test_window_matches_brute_force_matrix_form(shape, w):
+    B, Hq, Hkv, Tq, Tk, D = shape
+    q, k, v = rand_qkv(B, Hq, Hkv, Tq, Tk, D, seed=35)
+    ref = brute_force_attention(f64(q), f64(k), f64(v), window=w)
+    np.testing.assert_allclose(att(q, k, v, window=w), ref, rtol=0, atol=1e-12)
+
+
+def test_window_at_least_the_context_is_plain_causal():
+    q, k, v = rand_qkv(1, 4, 2, 6, 10, 8, seed=37)
+    full = att(q, k, v)
+    for w in (10, 11, 1000):
+        np.testing.assert_array_equal(att(q, k, v, window=w), full)
+    assert not np.array_equal(att(q, k, v, window=9), full)
+
+
+def test_window_suffix_consistency():
+    """The pages' suffix check also holds under a window."""
+    q, k, v = rand_qkv(2, 4, 2, 6, 6, 8, seed=39)
+    full = att(q, k, v, window=3)
+    np.testing.assert_array_equal(att(np.ascontiguousarray(q[:, :, -2:]), k, v, window=3), full[:, :, -2:])
