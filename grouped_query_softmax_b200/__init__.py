@@ -17,8 +17,9 @@ import ctypes
 import os
 
 __all__ = [
-    "GqaError", "gqa_attn_fwd", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
-    "gqa_attn_decode_num_splits", "gqa_attn_decode_static", "gqa_status_string", "gqa_get_device_error",
+    "GqaError", "gqa_attn_fwd", "gqa_attn_fwd_ex", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
+    "gqa_attn_decode_num_splits", "gqa_attn_decode_static", "gqa_attn_decode_ex",
+    "gqa_attn_decode_ex_workspace_bytes", "gqa_attn_decode_ex_num_splits", "gqa_status_string", "gqa_get_device_error",
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
@@ -46,6 +47,9 @@ _vp, _i32, _ll, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ct
 _lib.gqa_attn_fwd.restype = _i32
 _lib.gqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                               _ll, _ll, _ll, _ll, _f32, _vp]
+_lib.gqa_attn_fwd_ex.restype = _i32
+_lib.gqa_attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                 _ll, _ll, _ll, _ll, _f32, _i32, _vp]
 _lib.gqa_attn_decode_workspace_bytes.restype = _sz
 _lib.gqa_attn_decode_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.gqa_attn_decode_num_splits.restype = _i32
@@ -53,6 +57,13 @@ _lib.gqa_attn_decode_num_splits.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.gqa_attn_decode.restype = _i32
 _lib.gqa_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                  _ll, _ll, _ll, _ll, _f32, _i32, _vp, _sz, _vp]
+_lib.gqa_attn_decode_ex_workspace_bytes.restype = _sz
+_lib.gqa_attn_decode_ex_workspace_bytes.argtypes = [_i32] * 8
+_lib.gqa_attn_decode_ex_num_splits.restype = _i32
+_lib.gqa_attn_decode_ex_num_splits.argtypes = [_i32] * 8
+_lib.gqa_attn_decode_ex.restype = _i32
+_lib.gqa_attn_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                    _ll, _ll, _ll, _ll, _f32, _i32, _i32, _vp, _sz, _vp]
 _lib.gqa_attn_decode_static.restype = _i32
 _lib.gqa_attn_decode_static.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                         _ll, _ll, _ll, _ll, _f32, _i32, _vp]
@@ -82,6 +93,13 @@ def gqa_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
                              float(softmax_scale), stream)
 
 
+def gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                    softmax_scale=0.0, window=0, stream=None) -> int:
+    """C ``gqa_attn_fwd_ex``: ``gqa_attn_fwd`` with a sliding window (0 = causal only)."""
+    return _lib.gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                                float(softmax_scale), int(window), stream)
+
+
 def gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits=0) -> int:
     return int(_lib.gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits))
 
@@ -96,6 +114,23 @@ def gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb,
     """C ``gqa_attn_decode``; pointers are integers (device addresses). Returns the status."""
     return _lib.gqa_attn_decode(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
                                 float(softmax_scale), num_splits, workspace, workspace_bytes, stream)
+
+
+def gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window=0, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window, num_splits))
+
+
+def gqa_attn_decode_ex_num_splits(B, Hq, Hkv, Tq, Tk, D, window=0, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_ex_num_splits(B, Hq, Hkv, Tq, Tk, D, window, num_splits))
+
+
+def gqa_attn_decode_ex(q, k_cache, v_cache, o, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                       softmax_scale=0.0, window=0, num_splits=0, workspace=None, workspace_bytes=0,
+                       stream=None) -> int:
+    """C ``gqa_attn_decode_ex``: decode of 1 <= Tq <= 16 new queries per head, optional window."""
+    return _lib.gqa_attn_decode_ex(q, k_cache, v_cache, o, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb,
+                                   v_sh, float(softmax_scale), int(window), int(num_splits), workspace,
+                                   workspace_bytes, stream)
 
 
 def gqa_attn_decode_static(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh,
@@ -144,10 +179,11 @@ def _plane_strides(t, name):
     return t.stride(0), t.stride(1)
 
 
-def attn_fwd(q, k, v, *, Tk=None, scale=None, return_lse=False, out=None, stream=None):
+def attn_fwd(q, k, v, *, Tk=None, scale=None, window=0, return_lse=False, out=None, stream=None):
     """o = causal GQA attention of q [B,Hq,Tq,D] over k, v [B,Hkv,T_cap,D] (first Tk rows).
 
-    Query row i sits at position Tk - Tq + i. Returns o (bf16, [B,Hq,Tq,D]) and, if
+    Query row i sits at position Tk - Tq + i; ``window`` > 0 limits it to its
+    ``window`` most recent positions. Returns o (bf16, [B,Hq,Tq,D]) and, if
     ``return_lse``, the fp32 natural-log log-sum-exp [B,Hq,Tq].
     """
     torch = _torch()
@@ -167,39 +203,42 @@ def attn_fwd(q, k, v, *, Tk=None, scale=None, return_lse=False, out=None, stream
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
-    st = gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                      lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Tq, Tk, D,
-                      k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), _stream_handle(stream))
+    st = gqa_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Tq, Tk, D,
+                         k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), int(window),
+                         _stream_handle(stream))
     if st != GQA_OK:
-        raise GqaError(st, "gqa_attn_fwd")
+        raise GqaError(st, "gqa_attn_fwd_ex")
     return (out, lse) if return_lse else out
 
 
-def attn_decode(q, k_cache, v_cache, *, Tk=None, scale=None, num_splits=0, out=None,
+def attn_decode(q, k_cache, v_cache, *, Tk=None, scale=None, window=0, num_splits=0, out=None,
                 workspace=None, stream=None):
-    """One decode step: q [B,Hq,1,D] (or [B,Hq,D]) over the first Tk cached keys."""
+    """One decode step: q [B,Hq,Tq,D] (Tq <= 16; or [B,Hq,D] for Tq = 1) over the first Tk
+    cached keys; query row i sits at position Tk - Tq + i."""
     torch = _torch()
     for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
         _check_bf16_cuda(t, n)
     if not q.is_contiguous():
         raise ValueError("q must be contiguous")
     B, Hq, D = q.shape[0], q.shape[1], q.shape[-1]
-    if q.numel() != B * Hq * D:
-        raise ValueError("decode takes one query per (batch, head)")
+    Tq = q.shape[2] if q.dim() == 4 else 1
+    if q.numel() != B * Hq * Tq * D:
+        raise ValueError("q must be [B, Hq, Tq, D] or [B, Hq, D]")
     Hkv = k_cache.shape[1]
     Tk = k_cache.shape[2] if Tk is None else int(Tk)
     k_sb, k_sh = _plane_strides(k_cache, "k_cache")
     v_sb, v_sh = _plane_strides(v_cache, "v_cache")
     if out is None:
         out = torch.empty_like(q)
-    need = gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits)
+    need = gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window, num_splits)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = gqa_attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
-                         B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb, v_sh, float(scale or 0.0),
-                         int(num_splits), ws_ptr, ws_bytes, _stream_handle(stream))
+    st = gqa_attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                            B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh, float(scale or 0.0),
+                            int(window), int(num_splits), ws_ptr, ws_bytes, _stream_handle(stream))
     if st != GQA_OK:
-        raise GqaError(st, "gqa_attn_decode")
+        raise GqaError(st, "gqa_attn_decode_ex")
     return out

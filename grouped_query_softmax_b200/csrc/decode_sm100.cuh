@@ -1,15 +1,17 @@
-// Decode (T_q = 1) over a bf16 KV cache: split-KV partials + log-sum-exp combine.
+// Decode over a bf16 KV cache (T_q = 1, or a short chunk of T_q <= 16 new queries):
+// split-KV partials + log-sum-exp combine.
 //
-// The query of head a sits at position T_k - 1 and sees every cached key
-// ("注意力家族", section 最小语义实现: the suffix case with one query). Decode is
+// Query row i of head a sits at position T_k - T_q + i and sees keys up to it (for
+// T_q = 1 every cached key) -- "注意力家族", section 最小语义实现: the suffix case;
+// with a window it sees only its `window` most recent positions. Decode is
 // bound by the bytes of K/V it must stream ("注意力家族", section KV Cache 成本: the
 // cache is read again at every decode step; "Attention Architecture Evolution",
 // section Full Attention: decode is limited by memory bandwidth), so the kernel
 // reads every K/V byte of a KV head exactly once for all H_q/H_kv query heads that
 // share it ("A Visual Guide to Attention", section "How many KV heads?").
 //
-// Work unit = (split of the key axis, KV head g, batch b, chunk of 16 query heads of
-// group g). One producer warp streams 128-key K and V tiles with TMA (128-byte
+// Work unit = (split of the key axis, KV head g, batch b, chunk of 16 query rows of
+// group g, the G heads' T_q rows packed together). One producer warp streams 128-key K and V tiles with TMA (128-byte
 // swizzle) through a ring deep enough to keep >= 128 KB in flight per SM. Four
 // consumer warps each take 32 keys of every tile and keep their own running
 // (max, sum, O); scores and P.V use warp-level bf16 tensor-core MMAs with the query
@@ -25,21 +27,23 @@
 namespace gqa {
 
 constexpr int kDecKeys = 128;     // keys per streamed tile
-constexpr int kDecRows = 16;      // query heads per CTA (one m16 tile)
+constexpr int kDecRows = 16;      // query rows per CTA (one m16 tile)
 constexpr int kDecConsumers = 4;  // consumer warps
 constexpr int kDecThreads = 32 * (1 + kDecConsumers);
 
 struct DecParams {
-    int B, Hq, Hkv, Tk, G;
-    int n_hc;        // chunks of 16 query heads per group
+    int B, Hq, Hkv, Tq, Tk, G;
+    int n_hc;        // chunks of 16 query rows per group (a group has G * Tq rows)
     int splits;      // key-axis splits
     int blk_per_split;
+    int blk_first;   // first key block any row can see
     int n_blk;       // ceil(Tk / 128)
+    int window;      // > 0: each row sees only its `window` most recent positions
     float scale_log2;
-    const __nv_bfloat16* q;  // [B, Hq, D]
-    __nv_bfloat16* o;        // [B, Hq, D] (written when splits == 1)
-    float* ws_o;             // [splits, B, Hq, D] normalised partial outputs
-    float* ws_lse;           // [splits, B, Hq] log2-domain log-sum-exp
+    const __nv_bfloat16* q;  // [B, Hq, Tq, D]
+    __nv_bfloat16* o;        // [B, Hq, Tq, D] (written when splits == 1)
+    float* ws_o;             // [splits, B * Hq * Tq, D] normalised partial outputs
+    float* ws_lse;           // [splits, B * Hq * Tq] log2-domain log-sum-exp
     uint32_t* err;
     unsigned long long timeout_ns;
 };
@@ -93,11 +97,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int g = blockIdx.y / p.n_hc;
     const int hc = blockIdx.y - g * p.n_hc;
     const int b = blockIdx.z;
-    const int blk0 = split * p.blk_per_split;
+    const int blk0 = p.blk_first + split * p.blk_per_split;
     const int blk1 = min(blk0 + p.blk_per_split, p.n_blk);
     const int t_end = min(blk1 * kDecKeys, p.Tk);
-    const int head0 = g * p.G + hc * kDecRows;               // first query head of this CTA
-    const int nrows = min(kDecRows, p.G - hc * kDecRows);    // valid heads in the chunk
+    // Query rows of group g: the G heads' Tq rows each, contiguous in q ((a, i) order).
+    const int group_rows = p.G * p.Tq;
+    const int rbase = hc * kDecRows;                            // first row of this CTA
+    const int nrows = min(kDecRows, group_rows - rbase);        // valid rows in the chunk
+    const size_t row0 = ((size_t)b * p.Hq + (size_t)g * p.G) * p.Tq + rbase;  // flat row id
+    // rows see keys up to their own position (Tk - Tq + i) and, in a window, from
+    // position - window + 1; tiles touching either bound are masked element-wise
+    const int pos_min = p.Tk - p.Tq;
+    const int lo_max = p.window > 0 ? p.Tk - p.window : -1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -150,10 +161,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int cw = warp - 1;  // consumer index: keys [cw*32, cw*32+32) of every tile
         const int r_lo = lane >> 2;
         const int c2 = (lane & 3) * 2;
-        // Q fragments (A operand, rows = heads). Rows beyond the group are zero.
+        // Q fragments (A operand, rows = query rows). Rows beyond the group are zero.
         uint32_t qa[D / 16][4];
+        // absolute positions of this thread's two rows, and the first key they see
+        int rpos[2], rlo[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int rr = rbase + r_lo + 8 * h;
+            rpos[h] = p.Tk - p.Tq + rr % p.Tq;
+            rlo[h] = p.window > 0 ? rpos[h] - p.window + 1 : -1;
+        }
         {
-            const __nv_bfloat16* q0 = p.q + ((size_t)b * p.Hq + head0) * D;
+            const __nv_bfloat16* q0 = p.q + row0 * D;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
 #pragma unroll
@@ -197,14 +216,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     mma_bf16_16816(sacc[np * 2 + 1], qa[ks], b2, b3);
                 }
             }
-            // keys past the end of this split (or of the cache) do not exist
-            if (blk * kDecKeys + kDecKeys > t_end) {
+            // keys past the split's end, after the row's position or before its window
+            if (blk * kDecKeys + kDecKeys > min(t_end, pos_min + 1) || blk * kDecKeys < lo_max) {
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int key = blk * kDecKeys + cw * 32 + nt * 8 + c2 + (e & 1);
-                        if (key >= t_end) sacc[nt][e] = -INFINITY;
+                        const int h = e >> 1;
+                        if (key >= t_end || key > rpos[h] || key < rlo[h]) sacc[nt][e] = -INFINITY;
                     }
             }
             // ---- online softmax, one row half at a time
@@ -305,14 +325,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 lsum += bw[kDecRows + row] * sc;
                 acc += bw[2 * kDecRows + row * D + d] * sc;
             }
-            const int head = head0 + row;
-            const float val = acc / lsum;
+            const size_t frow = row0 + row;   // flat row id in [B * Hq * Tq]
+            // a row can see no key of this split (window, or keys past its position):
+            // its partial is 0 with log-sum-exp -inf, which the merge weighs by 0
+            const float val = lsum > 0.f ? acc / lsum : 0.f;
             if (p.splits == 1) {
-                p.o[((size_t)b * p.Hq + head) * D + d] = __float2bfloat16_rn(val);
+                p.o[frow * D + d] = __float2bfloat16_rn(val);
             } else {
-                const size_t prow = ((size_t)split * p.B + b) * p.Hq + head;
+                const size_t prow = (size_t)split * ((size_t)p.B * p.Hq * p.Tq) + frow;
                 p.ws_o[prow * D + d] = val;
-                if (d == 0) p.ws_lse[prow] = M + __log2f(lsum);
+                if (d == 0) p.ws_lse[prow] = lsum > 0.f ? M + __log2f(lsum) : -INFINITY;
             }
         }
     }

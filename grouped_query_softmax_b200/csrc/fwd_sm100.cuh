@@ -60,6 +60,7 @@ struct FwdParams {
     int per_level;   // work units per row level
     int units;       // total work units (grid-strided by the persistent CTAs)
     float scale_log2;
+    int window;      // > 0: each query sees only its `window` most recent positions
     __nv_bfloat16* o;
     float* lse;  // nullable
     uint32_t* err;
@@ -92,10 +93,12 @@ struct FwdSmem {
 };
 
 struct SubTile {
-    int head;       // query head a
-    int row0;       // first query row of the sub-tile
-    int n_kv;       // KV tiles to visit (0 = sub-tile absent)
-    int masked_from;  // first KV tile that crosses the diagonal
+    int head;         // query head a
+    int row0;         // first query row of the sub-tile
+    int j_begin;      // first KV tile to visit (> 0 only inside a sliding window)
+    int n_kv;         // KV tiles end (exclusive); the sub-tile visits [j_begin, n_kv) (n_kv 0 = absent)
+    int masked_from;  // first KV tile that crosses the causal diagonal
+    int lo_masked_end;  // KV tiles below this cross the lower edge of the window
 };
 
 __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& b, int& g,
@@ -123,6 +126,8 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
     g = st[0].head / p.G;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
+        st[s].j_begin = 0;
+        st[s].lo_masked_end = 0;
         if (st[s].row0 >= p.Tq) {
             st[s].n_kv = 0;
             st[s].masked_from = 0;
@@ -130,6 +135,14 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
             const int last = min(st[s].row0 + kFwdRows - 1, p.Tq - 1);
             st[s].n_kv = (off + last) / kFwdKeys + 1;
             st[s].masked_from = (off + st[s].row0 + 1) / kFwdKeys;
+            if (p.window > 0) {
+                // row positions P0..P1 see keys (P - w, P]: tiles before the first row's
+                // window are skipped, tiles before the last row's window start are masked
+                const int lo_first = off + st[s].row0 - p.window + 1;
+                const int lo_last = off + last - p.window + 1;
+                st[s].j_begin = lo_first > 0 ? lo_first / kFwdKeys : 0;
+                st[s].lo_masked_end = lo_last > 0 ? (lo_last + kFwdKeys - 1) / kFwdKeys : 0;
+            }
         }
     }
 }
@@ -217,6 +230,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 SubTile st[2];
                 fwd_decode_unit(p, u, b, g, st);
                 const int n_max = max(st[0].n_kv, st[1].n_kv);
+                const int jb = st[1].n_kv > 0 ? min(st[0].j_begin, st[1].j_begin) : st[0].j_begin;
                 // the previous unit's Q K^T products must be done before Q is replaced
                 if (q_loads > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->q_empty), (q_loads - 1) & 1u,
                                                             abort_flag, p.err, p.timeout_ns)))
@@ -228,7 +242,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         tma_load_4d(sQ + s * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64,
                                     st[s].row0, st[s].head, b);
                 ++q_loads;
-                for (int j = 0; j < n_max && ok; ++j) {
+                for (int j = jb; j < n_max && ok; ++j) {
                     for (int t = 0; t < 2; ++t) {
                         if (!(ok = mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
                                                      p.err, p.timeout_ns)))
@@ -312,6 +326,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 SubTile st[2];
                 fwd_decode_unit(p, u, b, g, st);
                 const int n_max = max(st[0].n_kv, st[1].n_kv);
+                // KV tiles jb .. n_max-1; sub-tile s uses tiles st[s].j_begin .. st[s].n_kv-1
+                const int jb = st[1].n_kv > 0 ? min(st[0].j_begin, st[1].j_begin) : st[0].j_begin;
+                auto in_range = [&](int s, int jj) { return jj >= st[s].j_begin && jj < st[s].n_kv; };
                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->q_full), q_uses & 1u, abort_flag, p.err,
                                              p.timeout_ns)))
                     break;
@@ -319,13 +336,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 int kslot;
                 if (!(ok = acquire(kslot))) break;
                 for (int s = 0; s < 2; ++s)
-                    if (st[s].n_kv > 0) {
+                    if (in_range(s, jb)) {
                         issue_qk(s, kslot);
                         tc_commit(smem_u32(&ctl->s_full[s]));
                     }
                 tc_commit(smem_u32(&ctl->empty[kslot]));
-                if (n_max == 1) tc_commit(smem_u32(&ctl->q_empty));
-                for (int j = 0; j < n_max && ok; ++j) {
+                if (n_max - jb == 1) tc_commit(smem_u32(&ctl->q_empty));
+                for (int j = jb; j < n_max && ok; ++j) {
                     int vslot;
                     if (!(ok = acquire(vslot))) break;
                     const bool next = j + 1 < n_max;
@@ -334,19 +351,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     int knext = -1;
                     if (next && !(ok = acquire(knext))) break;
                     for (int s = 0; s < 2 && ok; ++s) {
-                        if (j < st[s].n_kv) {
+                        if (in_range(s, j)) {
                             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full[s]), pph[s], abort_flag,
                                                          p.err, p.timeout_ns)))
                                 break;
                             pph[s] ^= 1u;
-                            if (j == 0 && o_uses[s] > 0) {
+                            if (j == st[s].j_begin && o_uses[s] > 0) {
                                 // the previous unit's epilogue must have read O_s
                                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->o_empty[s]), (o_uses[s] - 1) & 1u,
                                                              abort_flag, p.err, p.timeout_ns)))
                                     break;
                             }
                             tc_fence_after_sync();
-                            issue_pv(s, vslot, j > 0);
+                            issue_pv(s, vslot, j > st[s].j_begin);
                             if (j == st[s].n_kv - 1) {
                                 tc_commit(smem_u32(&ctl->o_full[s]));
                                 ++o_uses[s];
@@ -354,7 +371,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         }
                         if (s == 1) tc_commit(smem_u32(&ctl->empty[vslot]));
                         if (next) {
-                            if (j + 1 < st[s].n_kv) {
+                            if (in_range(s, j + 1)) {
                                 issue_qk(s, knext);
                                 tc_commit(smem_u32(&ctl->s_full[s]));
                             }
@@ -394,9 +411,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const SubTile me = st[s];
             if (me.n_kv == 0) continue;
             const int pos = off + me.row0 + r;  // absolute position of this query row
+            const int lo = pos - p.window + 1;  // first key inside the window (window > 0)
             float m = -INFINITY;  // running max of scaled scores (log2 units)
             float l = 0.f;        // running sum of exp2(score - m)
-            for (int j = 0; j < me.n_kv; ++j) {
+            for (int j = me.j_begin; j < me.n_kv; ++j) {
                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full[s]), sph, abort_flag, p.err,
                                              p.timeout_ns)))
                     break;
@@ -410,7 +428,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 reg_fence32(sr[1]);
                 tmem_ld32(tS + 64, sr[2]);
                 tmem_ld32(tS + 96, sr[3]);
-                const bool diag = j >= me.masked_from;
+                const bool diag = j >= me.masked_from || j < me.lo_masked_end;
                 // row max: eight independent chains of 3-input max, then a small tree; the
                 // first 64 columns are reduced while the last 64 are still loading
                 float mx[8];
@@ -429,12 +447,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 reg_fence32(sr[2]);
                 reg_fence32(sr[3]);
                 if (diag) {
-                    const int lim = pos - j * kFwdKeys;  // columns > lim are in the future
+                    // columns > lim are in the future; columns < lim_lo are before the window
+                    const int lim = pos - j * kFwdKeys;
+                    const int lim_lo = p.window > 0 ? lo - j * kFwdKeys : -1;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            if (c * 32 + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+                            if (c * 32 + e > lim || c * 32 + e < lim_lo) sr[c][e] = __float_as_uint(-INFINITY);
                         }
                 }
 #pragma unroll
@@ -453,7 +473,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const float alpha = refresh ? ex2_approx(m - m_new) : 1.f;
                 l *= alpha;
                 m = refresh ? m_new : m;
-                if (j > 0 && __any_sync(0xffffffffu, refresh)) {
+                if (j > me.j_begin && __any_sync(0xffffffffu, refresh)) {
                     // O_s has absorbed all earlier P V products (their completion is
                     // ordered before S_j's commit); rescale this row in place.
 #pragma unroll 1

@@ -83,31 +83,51 @@ int device_sm_count() {
     return sms;
 }
 
+constexpr int kMaxDecodeRows = 16;  // query rows per head the decode path takes (T_q)
+
 struct SplitPlan {
-    int splits, blk_per_split, n_blk;
+    int splits, blk_per_split, blk_first, n_blk;
 };
 
-SplitPlan plan_splits(int B, int Hq, int Hkv, int Tk, int requested) {
+// Key blocks [blk_first, n_blk) hold every key some query row can see: with a window
+// the rows of a chunk (positions Tk-Tq .. Tk-1) see nothing before Tk - Tq - window + 1.
+SplitPlan plan_splits(int B, int Hq, int Hkv, int Tq, int Tk, int window, int requested) {
     SplitPlan sp{};
     sp.n_blk = (Tk + gqa::kTileKeys - 1) / gqa::kTileKeys;
+    const int key_lo = window > 0 ? std::max(0, Tk - Tq - window + 1) : 0;
+    sp.blk_first = key_lo / gqa::kTileKeys;
+    const int n_range = sp.n_blk - sp.blk_first;
     const int G = Hq / Hkv;
-    const long long units = (long long)B * Hkv * ((G + 15) / 16);
+    const long long units = (long long)B * Hkv * ((G * Tq + 15) / 16);
     int want = requested;
     if (want <= 0) {
         // about four waves of one CTA per SM, each split at least 8 tiles (1024 keys)
         const long long target = 4LL * device_sm_count();
         want = (int)std::min<long long>((target + units - 1) / units, 1 << 20);
-        want = std::min(want, std::max(1, sp.n_blk / 8));
+        want = std::min(want, std::max(1, n_range / 8));
     }
-    want = std::max(1, std::min(want, sp.n_blk));
-    sp.blk_per_split = (sp.n_blk + want - 1) / want;
-    sp.splits = (sp.n_blk + sp.blk_per_split - 1) / sp.blk_per_split;  // no empty split
+    want = std::max(1, std::min(want, n_range));
+    sp.blk_per_split = (n_range + want - 1) / want;
+    sp.splits = (n_range + sp.blk_per_split - 1) / sp.blk_per_split;  // no empty split
     return sp;
 }
 
-size_t ws_lse_offset(int splits, int B, int Hq, int D) {
-    const size_t o_bytes = (size_t)splits * B * Hq * D * sizeof(float);
+size_t ws_lse_offset(int splits, long long rows, int D) {
+    const size_t o_bytes = (size_t)splits * rows * D * sizeof(float);
     return (o_bytes + 255) & ~(size_t)255;
+}
+
+size_t ws_bytes_for(const SplitPlan& sp, long long rows, int D) {
+    if (sp.splits == 1) return 0;
+    return ws_lse_offset(sp.splits, rows, D) + (size_t)sp.splits * rows * sizeof(float);
+}
+
+gqa_status check_decode(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window) {
+    gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
+    if (st != GQA_OK) return st;
+    if (window < 0) return GQA_ERR_INVALID_ARGUMENT;
+    if (Tq > kMaxDecodeRows) return GQA_ERR_UNSUPPORTED;  // longer chunks: gqa_attn_fwd_ex
+    return GQA_OK;
 }
 
 }  // namespace
@@ -129,8 +149,17 @@ const char* gqa_status_string(gqa_status s) {
 gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh,
                         long long v_sb, long long v_sh, float softmax_scale, void* stream) {
+    return gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                           softmax_scale, 0, stream);
+}
+
+gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh,
+                           long long v_sb, long long v_sh, float softmax_scale, int window,
+                           void* stream) {
     gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
     if (st != GQA_OK) return st;
+    if (window < 0) return GQA_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GQA_ERR_INVALID_ARGUMENT;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
     if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
@@ -143,54 +172,75 @@ gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
     if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.window = window >= Tk ? 0 : window;  // a window covering every key is plain causal
     a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
     a.o = o;
     a.lse = lse;
     return gqa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
-int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
-    if (check_common(B, Hq, Hkv, 1, Tk, D) != GQA_OK) return 0;
-    return plan_splits(B, Hq, Hkv, Tk, num_splits).splits;
+int gqa_attn_decode_ex_num_splits(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window,
+                                  int num_splits) {
+    if (check_decode(B, Hq, Hkv, Tq, Tk, D, window) != GQA_OK) return 0;
+    return plan_splits(B, Hq, Hkv, Tq, Tk, window, num_splits).splits;
 }
 
-size_t gqa_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
-    if (check_common(B, Hq, Hkv, 1, Tk, D) != GQA_OK) return 0;
-    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tk, num_splits);
-    if (sp.splits == 1) return 0;
-    return ws_lse_offset(sp.splits, B, Hq, D) + (size_t)sp.splits * B * Hq * sizeof(float);
+size_t gqa_attn_decode_ex_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window,
+                                          int num_splits) {
+    if (check_decode(B, Hq, Hkv, Tq, Tk, D, window) != GQA_OK) return 0;
+    return ws_bytes_for(plan_splits(B, Hq, Hkv, Tq, Tk, window, num_splits), (long long)B * Hq * Tq, D);
 }
 
-gqa_status gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, int B,
-                           int Hq, int Hkv, int Tk, int D, long long k_sb, long long k_sh,
-                           long long v_sb, long long v_sh, float softmax_scale, int num_splits,
-                           void* workspace, size_t workspace_bytes, void* stream) {
-    gqa_status st = check_common(B, Hq, Hkv, 1, Tk, D);
+gqa_status gqa_attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, void* o, int B,
+                              int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh,
+                              long long v_sb, long long v_sh, float softmax_scale, int window,
+                              int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+    gqa_status st = check_decode(B, Hq, Hkv, Tq, Tk, D, window);
     if (st != GQA_OK) return st;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return GQA_ERR_INVALID_ARGUMENT;
     if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
     if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
     if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
-    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tk, num_splits);
+    if (window >= Tk) window = 0;  // a window covering every key is plain causal
+    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tq, Tk, window, num_splits);
+    const long long rows = (long long)B * Hq * Tq;
     gqa::DecLaunch a{};
     if (sp.splits > 1) {
-        const size_t need = ws_lse_offset(sp.splits, B, Hq, D) + (size_t)sp.splits * B * Hq * sizeof(float);
+        const size_t need = ws_bytes_for(sp, rows, D);
         if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
             return GQA_ERR_WORKSPACE;
         a.ws_o = static_cast<float*>(workspace);
-        a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_lse_offset(sp.splits, B, Hq, D));
+        a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_lse_offset(sp.splits, rows, D));
     }
     if ((st = make_map(&a.tm_k, k_cache, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
     if ((st = make_map(&a.tm_v, v_cache, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
-    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tk = Tk; a.D = D;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.window = window;
     a.splits = sp.splits;
     a.blk_per_split = sp.blk_per_split;
+    a.blk_first = sp.blk_first;
     a.n_blk = sp.n_blk;
     a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
     a.q = q;
     a.o = o;
     return gqa::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
+    return gqa_attn_decode_ex_num_splits(B, Hq, Hkv, 1, Tk, D, 0, num_splits);
+}
+
+size_t gqa_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Tk, int D, int num_splits) {
+    return gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, 1, Tk, D, 0, num_splits);
+}
+
+gqa_status gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, int B,
+                           int Hq, int Hkv, int Tk, int D, long long k_sb, long long k_sh,
+                           long long v_sb, long long v_sh, float softmax_scale, int num_splits,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    return gqa_attn_decode_ex(q, k_cache, v_cache, o, B, Hq, Hkv, 1, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                              softmax_scale, 0, num_splits, workspace, workspace_bytes, stream);
 }
 
 gqa_status gqa_get_device_error(void* stream) {

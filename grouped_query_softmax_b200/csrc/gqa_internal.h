@@ -11,6 +11,7 @@ namespace gqa {
 struct FwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v;
     int B, Hq, Hkv, Tq, Tk, D;
+    int window;  // 0: causal; > 0: sliding window of that many positions
     float scale;
     void* o;
     float* lse;
@@ -18,8 +19,9 @@ struct FwdLaunch {
 
 struct DecLaunch {
     CUtensorMap tm_k, tm_v;
-    int B, Hq, Hkv, Tk, D;
-    int splits, blk_per_split, n_blk;
+    int B, Hq, Hkv, Tq, Tk, D;
+    int window;
+    int splits, blk_per_split, blk_first, n_blk;
     float scale;
     const void* q;
     void* o;

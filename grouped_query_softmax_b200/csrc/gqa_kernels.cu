@@ -40,6 +40,7 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
         units = (long long)p.per_level * ((p.n_qt + 1) / 2);
     }
     p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.window = a.window;
     p.o = static_cast<__nv_bfloat16*>(a.o);
     p.lse = a.lse;
     p.err = device_error_ptr();
@@ -77,12 +78,15 @@ static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
     p.B = a.B;
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
+    p.Tq = a.Tq;
     p.Tk = a.Tk;
     p.G = a.Hq / a.Hkv;
-    p.n_hc = (p.G + kDecRows - 1) / kDecRows;
+    p.n_hc = (p.G * a.Tq + kDecRows - 1) / kDecRows;
     p.splits = a.splits;
     p.blk_per_split = a.blk_per_split;
+    p.blk_first = a.blk_first;
     p.n_blk = a.n_blk;
+    p.window = a.window;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.o = static_cast<__nv_bfloat16*>(a.o);
@@ -99,7 +103,7 @@ static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
     gqa_decode_sm100_kernel<D><<<grid, kDecThreads, smem, stream>>>(a.tm_k, a.tm_v, p);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
-    const int rows = a.B * a.Hq;
+    const int rows = a.B * a.Hq * a.Tq;
     gqa_decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
         a.ws_o, a.ws_lse, static_cast<__nv_bfloat16*>(a.o), rows, a.splits);
     return cudaGetLastError();

@@ -79,6 +79,19 @@ GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, voi
                         float softmax_scale, void* stream);
 
 /*
+ * gqa_attn_fwd with a sliding window: window > 0 restricts the query at position p to
+ * its `window` most recent positions, keys j with p - window < j <= p (itself
+ * included) -- "A Visual Guide to Attention", section "Which positions are visible?"
+ * (sliding-window attention; GQA combined with it as in Mistral 7B, section "Read the
+ * data path"). KV tiles wholly outside every row's window are never loaded.
+ * window = 0 is plain causal attention; window < 0 is GQA_ERR_INVALID_ARGUMENT.
+ */
+GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Tq, int Tk, int D,
+                                   long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                                   float softmax_scale, int window, void* stream);
+
+/*
  * Decode (T_q = 1): the query of each (b, a) sits at position T_k - 1 and sees all
  * T_k cached keys ("注意力家族", section 最小语义实现: the suffix case with one
  * query). The KV cache is split into num_splits key ranges; each range yields a
@@ -125,6 +138,31 @@ GQA_API gqa_status gqa_attn_decode_static(const void* q, const void* k_cache, co
                                           long long k_sb, long long k_sh, long long v_sb,
                                           long long v_sh, float softmax_scale, int num_splits,
                                           void* stream);
+
+/*
+ * Decode of a short chunk of new queries, optionally in a sliding window: T_q in
+ * [1, 16] query rows per head at positions T_k - T_q .. T_k - 1 (speculative or
+ * verification chunks; "注意力家族", section 最小语义实现 -- the suffix case with
+ * query positions starting at T_k - T_q), each seeing keys up to its own position and,
+ * if window > 0, only its `window` most recent positions. The G * T_q rows of a KV
+ * head are packed into the same tensor-core tiles, so the cache is still read once
+ * per KV head.
+ *
+ *   q, o   bf16 [B, Hq, Tq, D], contiguous. Other arguments as gqa_attn_decode.
+ *   T_q > 16 returns GQA_ERR_UNSUPPORTED (use gqa_attn_fwd_ex); window < 0 returns
+ *   GQA_ERR_INVALID_ARGUMENT. The workspace is sized by
+ *   gqa_attn_decode_ex_workspace_bytes with the same arguments.
+ * gqa_attn_decode(...) is gqa_attn_decode_ex(..., Tq = 1, ..., window = 0, ...).
+ */
+GQA_API size_t gqa_attn_decode_ex_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D,
+                                                  int window, int num_splits);
+GQA_API int gqa_attn_decode_ex_num_splits(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window,
+                                          int num_splits);
+GQA_API gqa_status gqa_attn_decode_ex(const void* q, const void* k_cache, const void* v_cache,
+                                      void* o, int B, int Hq, int Hkv, int Tq, int Tk, int D,
+                                      long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                                      float softmax_scale, int window, int num_splits,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* The split count gqa_attn_decode will use for these arguments (num_splits 0 = auto). */
 GQA_API int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits);
