@@ -104,6 +104,7 @@ class Workload:
     D: int
     q_pow2: int = 0      # Q multiplied by 2**q_pow2 after bf16 rounding
     seed: int = 0
+    window: int = 0      # sliding window (0 = plain causal); a mask setting, not data
 
     @property
     def q_shape(self):
@@ -131,10 +132,17 @@ GQA_DECODE = Workload("GQA decode B64 Hq32 Hkv8 Tk32768 D128", 64, 32, 8, 1, 327
 MHA_SUFFIX = Workload("MHA suffix B8 H16 Tq512 at 7680 over Tk8192 D128 Qx4", 8, 16, 16, 512, 8192, 128,
                       q_pow2=2)
 
+# Workloads of the extension rows (sliding window, short decode chunks).
+SWA_PREFILL = Workload("GQA sliding-window prefill B4 Hq32 Hkv8 T4096 W1024 D128", 4, 32, 8, 4096, 4096,
+                       128, window=1024)
+CHUNK_DECODE = Workload("GQA verify chunk B64 Hq32 Hkv8 Tq4 Tk32768 D128", 64, 32, 8, 4, 32768, 128)
+
 WORKLOADS = {
     "tiny": TINY,
     "gqa_prefill": GQA_PREFILL,
     "mqa_long": MQA_LONG,
     "gqa_decode": GQA_DECODE,
     "mha_suffix": MHA_SUFFIX,
+    "swa_prefill": SWA_PREFILL,
+    "chunk_decode": CHUNK_DECODE,
 }

@@ -21,14 +21,14 @@ def _rows_to_f32(bits_flat, rows, D):
     return gi.bf16_bits_to_f32(bits_flat.reshape(-1, D)[rows]).astype(np.float64)
 
 
-@pytest.mark.parametrize("name", ["tiny", "gqa_prefill", "mqa_long", "mha_suffix"])
+@pytest.mark.parametrize("name", ["tiny", "gqa_prefill", "mqa_long", "mha_suffix", "swa_prefill"])
 def test_prefill_workload_full_size(name):
     torch = torch_mod()
     import grouped_query_softmax_b200 as gqa
     w = gi.WORKLOADS[name]
     q, k, v = w.make()
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
-    o = gqa.attn_fwd(qd, kd, vd)
+    o = gqa.attn_fwd(qd, kd, vd, window=w.window)
     torch.cuda.synchronize()
     assert gqa.gqa_get_device_error() == gqa.GQA_OK
     out_bits = bits_of(o)
@@ -38,7 +38,7 @@ def test_prefill_workload_full_size(name):
     else:
         rows = sample_rows(w.B, w.Hq, w.Tq, 4096, seed=1)
         assert len(rows) >= 4096
-    ref = oracle.attention_rows(q, k, v, rows)
+    ref = oracle.attention_rows(q, k, v, rows, window=w.window)
     assert_parity(_rows_to_f32(out_bits, rows, w.D), ref, f"{name} ({len(rows)} rows)")
     if name == "gqa_prefill":
         # run-to-run determinism of the full output
@@ -47,17 +47,18 @@ def test_prefill_workload_full_size(name):
         np.testing.assert_array_equal(bits_of(o2), out_bits)
 
 
-def test_decode_workload_full_size():
+@pytest.mark.parametrize("name", ["gqa_decode", "chunk_decode"])
+def test_decode_workload_full_size(name):
     torch = torch_mod()
     import grouped_query_softmax_b200 as gqa
-    w = gi.WORKLOADS["gqa_decode"]           # B64 Hq32 Hkv8, 32768 cached keys: 8 GiB of K/V
+    w = gi.WORKLOADS[name]                   # B64 Hq32 Hkv8, 32768 cached keys: 8 GiB of K/V
     q, k, v = w.make()
     kd = to_dev(k)
     vd = to_dev(v)
     qd = to_dev(q)
-    o = gqa.attn_decode(qd, kd, vd)          # automatic split count, as the bench runs it
+    o = gqa.attn_decode(qd, kd, vd, window=w.window)   # automatic split count, as the bench runs it
     torch.cuda.synchronize()
     assert gqa.gqa_get_device_error() == gqa.GQA_OK
-    rows = np.arange(w.B * w.Hq)
-    ref = oracle.attention_rows(q, k, v, rows)
-    assert_parity(_rows_to_f32(bits_of(o), rows, w.D), ref, "gqa_decode (all rows)")
+    rows = np.arange(w.B * w.Hq * w.Tq)
+    ref = oracle.attention_rows(q, k, v, rows, window=w.window)
+    assert_parity(_rows_to_f32(bits_of(o), rows, w.D), ref, f"{name} (all rows)")
