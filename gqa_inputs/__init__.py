@@ -24,6 +24,8 @@ _SRC = os.path.join(_HERE, "gen.c")
 _LIB = os.path.join(_HERE, "libgqa_inputs.so")
 
 TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
+# streams of the integer draws: query-chunk lengths, cached-prefix lengths, page order
+STREAM_LEN, STREAM_PREFIX, STREAM_PAGES = 3, 4, 5
 
 
 def build(force: bool = False) -> str:
@@ -47,6 +49,9 @@ def _load():
                                             ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int]
         lib.gqa_gen_key.restype = ctypes.c_uint64
         lib.gqa_gen_key.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
+        lib.gqa_gen_words.restype = None
+        lib.gqa_gen_words.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint64,
+                                      ctypes.c_uint64, ctypes.c_void_p]
         _lib = lib
     return _lib
 
@@ -69,6 +74,27 @@ def normal_bf16(seed: int, tensor_id: int, shape, start: int = 0, threads: int |
     _load().gqa_gen_normal_bf16(int(seed), int(tensor_id), int(start), n,
                                 out.ctypes.data, int(threads or default_threads()))
     return out
+
+
+def words(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
+    """Raw 64-bit words [start, start + n) of stream (seed, stream)."""
+    out = np.empty(int(n), dtype=np.uint64)
+    if n:
+        _load().gqa_gen_words(int(seed), int(stream), int(start), int(n), out.ctypes.data)
+    return out
+
+
+def uniform_ints(seed: int, stream: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """n integers in [lo, hi]: lo + word mod (hi - lo + 1) (int64)."""
+    if hi < lo:
+        raise ValueError("empty range")
+    w = words(seed, stream, n)
+    return (lo + (w % np.uint64(hi - lo + 1)).astype(np.int64)).astype(np.int64)
+
+
+def permutation(seed: int, stream: int, n: int) -> np.ndarray:
+    """A permutation of 0..n-1: the stable argsort of n words (int64)."""
+    return np.argsort(words(seed, stream, n), kind="stable").astype(np.int64)
 
 
 def bf16_bits_to_f32(u16: np.ndarray) -> np.ndarray:
@@ -145,4 +171,106 @@ WORKLOADS = {
     "mha_suffix": MHA_SUFFIX,
     "swa_prefill": SWA_PREFILL,
     "chunk_decode": CHUNK_DECODE,
+}
+
+
+def cu_from_lengths(lengths) -> np.ndarray:
+    """Sequence boundaries [0, l0, l0 + l1, ...] (int32) of packed sequences."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """Packed sequences of a variable length (chunked prefill of a serving step).
+
+    Sequence s has a new chunk of L_q(s) query tokens ~ U[q_lo, q_hi] after a cached
+    prefix of P(s) ~ U[prefix_lo, prefix_hi] tokens, so it attends over
+    L_k(s) = P(s) + L_q(s) keys. Q, K and V are token-major, [total, H, D] (the packed
+    layout of serving engines); every value is iid N(0,1) bf16 from the same streams
+    as the dense workloads."""
+    name: str
+    S: int
+    Hq: int
+    Hkv: int
+    D: int
+    q_lo: int
+    q_hi: int
+    prefix_lo: int = 0
+    prefix_hi: int = 0
+    seed: int = 0
+    window: int = 0
+
+    def lengths(self):
+        lq = uniform_ints(self.seed, STREAM_LEN, self.S, self.q_lo, self.q_hi)
+        if self.prefix_hi > 0:
+            pre = uniform_ints(self.seed, STREAM_PREFIX, self.S, self.prefix_lo, self.prefix_hi)
+        else:
+            pre = np.zeros(self.S, dtype=np.int64)
+        return lq, lq + pre
+
+    def make(self, threads: int | None = None):
+        """(q, k, v, cu_q, cu_k): token-major bf16 bit arrays and int32 boundaries."""
+        lq, lk = self.lengths()
+        cu_q, cu_k = cu_from_lengths(lq), cu_from_lengths(lk)
+        q = normal_bf16(self.seed, TENSOR_Q, (int(cu_q[-1]), self.Hq, self.D), threads=threads)
+        k = normal_bf16(self.seed, TENSOR_K, (int(cu_k[-1]), self.Hkv, self.D), threads=threads)
+        v = normal_bf16(self.seed, TENSOR_V, (int(cu_k[-1]), self.Hkv, self.D), threads=threads)
+        return q, k, v, cu_q, cu_k
+
+
+@dataclass(frozen=True)
+class PagedDecodeWorkload:
+    """Decode over a paged KV cache with a per-sequence cache length.
+
+    Sequence b has L(b) ~ U[len_lo, len_hi] cached tokens (its T_q new queries are the
+    last T_q of them) held in ceil(L(b) / page) pages of `page` tokens. The pool holds
+    exactly the pages in use, in a seeded random order (a fragmented cache), laid out
+    [pages, page, H_kv, D] (token-major inside a page); block_table[b, i] is the pool
+    page of the sequence's i-th page, -1 past its last page."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    len_lo: int
+    len_hi: int
+    page: int
+    Tq: int = 1
+    seed: int = 0
+    window: int = 0
+
+    def lengths(self):
+        return uniform_ints(self.seed, STREAM_LEN, self.B, self.len_lo, self.len_hi)
+
+    def make(self, threads: int | None = None):
+        """(q, k_pool, v_pool, lengths, block_table)."""
+        lens = self.lengths()
+        n_pages = (lens + self.page - 1) // self.page
+        total = int(n_pages.sum())
+        order = permutation(self.seed, STREAM_PAGES, total)
+        width = int(n_pages.max())
+        table = np.full((self.B, width), -1, dtype=np.int32)
+        at = 0
+        for b in range(self.B):
+            table[b, :n_pages[b]] = order[at:at + n_pages[b]]
+            at += int(n_pages[b])
+        q = normal_bf16(self.seed, TENSOR_Q, (self.B, self.Hq, self.Tq, self.D), threads=threads)
+        k = normal_bf16(self.seed, TENSOR_K, (total, self.page, self.Hkv, self.D), threads=threads)
+        v = normal_bf16(self.seed, TENSOR_V, (total, self.page, self.Hkv, self.D), threads=threads)
+        return q, k, v, lens.astype(np.int32), table
+
+
+# Workloads of the variable-length row.
+VARLEN_PREFILL = VarlenWorkload("GQA packed varlen prefill S16 chunks U[256,8192] Hq32 Hkv8 D128",
+                                16, 32, 8, 128, 256, 8192)
+CHUNKED_PREFILL = VarlenWorkload("GQA chunked prefill S32 chunks U[128,2048] after prefixes U[0,8192] "
+                                 "Hq32 Hkv8 D128", 32, 32, 8, 128, 128, 2048, 0, 8192)
+PAGED_DECODE = PagedDecodeWorkload("GQA paged decode B64 Hq32 Hkv8 D128 lengths U[4096,32768] page 64",
+                                   64, 32, 8, 128, 4096, 32768, 64)
+
+VARLEN_WORKLOADS = {
+    "varlen_prefill": VARLEN_PREFILL,
+    "chunked_prefill": CHUNKED_PREFILL,
+    "paged_decode": PAGED_DECODE,
 }

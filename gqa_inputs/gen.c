@@ -127,3 +127,10 @@ int gqa_gen_normal_bf16(uint64_t seed, uint32_t tensor_id, uint64_t start, uint6
         if (joined[t]) pthread_join(th[t], NULL);
     return 0;
 }
+
+/* Raw words word(start) .. word(start+count-1) of stream (seed, tensor_id): the
+ * integer draws of the recipe (sequence lengths, page assignments) use these. */
+void gqa_gen_words(uint64_t seed, uint32_t tensor_id, uint64_t start, uint64_t count, uint64_t* out) {
+    uint64_t key = gqa_gen_key(seed, tensor_id);
+    for (uint64_t i = 0; i < count; ++i) out[i] = mix64(key + (start + i + 1) * GQA_GOLDEN);
+}

@@ -48,3 +48,29 @@ def test_workload_shapes():
     t = gi.TINY
     q, k, v = t.make(threads=2)
     assert q.shape == (2, 4, 128, 64) and k.shape == (2, 2, 128, 64) and v.dtype == np.uint16
+
+
+def test_integer_draws_are_seeded_and_in_range():
+    a = gi.uniform_ints(0, gi.STREAM_LEN, 1000, 256, 8192)
+    np.testing.assert_array_equal(a, gi.uniform_ints(0, gi.STREAM_LEN, 1000, 256, 8192))
+    assert a.min() >= 256 and a.max() <= 8192 and len(set(a.tolist())) > 900
+    assert not np.array_equal(a, gi.uniform_ints(1, gi.STREAM_LEN, 1000, 256, 8192))
+    p = gi.permutation(0, gi.STREAM_PAGES, 777)
+    np.testing.assert_array_equal(np.sort(p), np.arange(777))
+    w = gi.words(3, 4, 10)
+    np.testing.assert_array_equal(w[4:], gi.words(3, 4, 6, start=4))
+
+
+def test_varlen_and_paged_workload_recipes():
+    w = gi.WORKLOADS.get("tiny")
+    assert w is not None
+    vw = gi.VARLEN_WORKLOADS["chunked_prefill"]
+    lq, lk = vw.lengths()
+    assert (lq >= vw.q_lo).all() and (lq <= vw.q_hi).all() and (lk >= lq).all()
+    pw = gi.PagedDecodeWorkload("t", 3, 4, 2, 8, 5, 40, 16)
+    q, k, v, lens, table = pw.make()
+    n_pages = (lens + 15) // 16
+    assert k.shape == (int(n_pages.sum()), 16, 2, 8) and q.shape == (3, 4, 1, 8)
+    used = np.sort(np.concatenate([table[b, :n_pages[b]] for b in range(3)]))
+    np.testing.assert_array_equal(used, np.arange(int(n_pages.sum())))   # every page once
+    assert all((table[b, n_pages[b]:] == -1).all() for b in range(3))
