@@ -21,6 +21,8 @@ __all__ = [
     "gqa_attn_decode_num_splits", "gqa_attn_decode_static", "gqa_attn_decode_ex",
     "gqa_attn_decode_ex_workspace_bytes", "gqa_attn_decode_ex_num_splits", "gqa_status_string", "gqa_get_device_error",
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
+    "GqaLayout", "gqa_attn_fwd_varlen", "gqa_attn_fwd_varlen_workspace_bytes", "gqa_attn_decode_varlen",
+    "attn_fwd_varlen", "attn_decode_varlen",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
 ]
@@ -67,6 +69,20 @@ _lib.gqa_attn_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, 
 _lib.gqa_attn_decode_static.restype = _i32
 _lib.gqa_attn_decode_static.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                         _ll, _ll, _ll, _ll, _f32, _i32, _vp]
+
+
+class GqaLayout(ctypes.Structure):
+    """C ``gqa_layout``: element strides (batch, head, row) of a bf16 operand; d is contiguous."""
+    _fields_ = [("sb", _ll), ("sh", _ll), ("st", _ll)]
+
+
+_lay = ctypes.POINTER(GqaLayout)
+_lib.gqa_attn_fwd_varlen_workspace_bytes.restype = _sz
+_lib.gqa_attn_fwd_varlen_workspace_bytes.argtypes = [_i32] * 4
+_lib.gqa_attn_fwd_varlen.restype = _i32
+_lib.gqa_attn_fwd_varlen.argtypes = ([_vp] * 9 + [_i32] * 7 + [_lay] * 4 + [_f32, _i32, _vp, _sz, _vp])
+_lib.gqa_attn_decode_varlen.restype = _i32
+_lib.gqa_attn_decode_varlen.argtypes = ([_vp] * 6 + [_i32] * 9 + [_lay] * 2 + [_f32, _i32, _i32, _vp, _sz, _vp])
 _lib.gqa_status_string.restype = ctypes.c_char_p
 _lib.gqa_status_string.argtypes = [_i32]
 _lib.gqa_get_device_error.restype = _i32
@@ -139,6 +155,41 @@ def gqa_attn_decode_static(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh
     instead of a caller workspace, for callers that cannot allocate device memory."""
     return _lib.gqa_attn_decode_static(q, k_cache, v_cache, o, B, Hq, Hkv, Tk, D, k_sb, k_sh, v_sb,
                                        v_sh, float(softmax_scale), num_splits, stream)
+
+
+def _layout(x):
+    if isinstance(x, GqaLayout):
+        return x
+    sb, sh, st = x
+    return GqaLayout(int(sb), int(sh), int(st))
+
+
+def gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q) -> int:
+    return int(_lib.gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q))
+
+
+def gqa_attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, seqlens_q, seqlens_k, S, Hq, Hkv,
+                        D, rows_q, rows_k, max_seqlen_q, q_layout, k_layout, v_layout, o_layout,
+                        softmax_scale=0.0, window=0, workspace=None, workspace_bytes=0,
+                        stream=None) -> int:
+    """C ``gqa_attn_fwd_varlen``; layouts are GqaLayout or (sb, sh, st) tuples in elements."""
+    lq, lk, lv, lo = (_layout(x) for x in (q_layout, k_layout, v_layout, o_layout))
+    return _lib.gqa_attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, seqlens_q, seqlens_k,
+                                    S, Hq, Hkv, D, rows_q, rows_k, max_seqlen_q, ctypes.byref(lq),
+                                    ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
+                                    float(softmax_scale), int(window), workspace, workspace_bytes, stream)
+
+
+def gqa_attn_decode_varlen(q, k_cache, v_cache, o, seqlens_k, block_table, page_size, num_pages,
+                           max_pages, B, Hq, Hkv, Tq, max_seqlen_k, D, k_layout, v_layout,
+                           softmax_scale=0.0, window=0, num_splits=0, workspace=None, workspace_bytes=0,
+                           stream=None) -> int:
+    """C ``gqa_attn_decode_varlen``: decode over per-sequence cache lengths, contiguous or paged."""
+    lk, lv = _layout(k_layout), _layout(v_layout)
+    return _lib.gqa_attn_decode_varlen(q, k_cache, v_cache, o, seqlens_k, block_table, page_size,
+                                       num_pages, max_pages, B, Hq, Hkv, Tq, max_seqlen_k, D,
+                                       ctypes.byref(lk), ctypes.byref(lv), float(softmax_scale),
+                                       int(window), int(num_splits), workspace, workspace_bytes, stream)
 
 
 def gqa_status_string(status: int) -> str:
@@ -241,4 +292,145 @@ def attn_decode(q, k_cache, v_cache, *, Tk=None, scale=None, window=0, num_split
                             int(window), int(num_splits), ws_ptr, ws_bytes, _stream_handle(stream))
     if st != GQA_OK:
         raise GqaError(st, "gqa_attn_decode_ex")
+    return out
+
+
+def _side_layout(t, name):
+    """(packed?, rows, H, layout) of a varlen operand: packed [rows, H, D] or padded [S, H, rows, D]."""
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name}: the last (D) axis must be contiguous")
+    if t.dim() == 3:
+        return True, t.shape[0], t.shape[1], (0, t.stride(1), t.stride(0))
+    if t.dim() == 4:
+        return False, t.shape[2], t.shape[1], (t.stride(0), t.stride(1), t.stride(2))
+    raise ValueError(f"{name} must be packed [rows, H, D] or padded [S, H, rows, D]")
+
+
+def _ptr(t):
+    return t.data_ptr() if t is not None else None
+
+
+def _int32_cuda(t, name):
+    torch = _torch()
+    if t is None:
+        return None
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous int32 CUDA tensor")
+    return t
+
+
+def attn_fwd_varlen(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, seqlens_q=None, seqlens_k=None,
+                    max_seqlen_q=None, scale=None, window=0, return_lse=False, out=None, workspace=None,
+                    stream=None):
+    """S independent causal GQA problems of different lengths in one call.
+
+    Each side is packed, a 3-D [rows, H, D] tensor (any row/head strides, so token-major
+    [total, H, D] and a transposed head-major buffer both work) with int32 boundaries
+    ``cu_seqlens_*`` [S + 1], or padded, a 4-D [S, H, rows, D] tensor with optional
+    lengths ``seqlens_*`` [S]. Sequence s's L_q query rows sit at positions L_k - L_q ..
+    L_k - 1 of its own keys. Returns o shaped like q (rows of no sequence untouched)
+    and, with ``return_lse``, the fp32 LSE [Hq, rows_q] (packed) or [S, Hq, rows_q].
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_bf16_cuda(t, n)
+    cu_q, cu_k = _int32_cuda(cu_seqlens_q, "cu_seqlens_q"), _int32_cuda(cu_seqlens_k, "cu_seqlens_k")
+    len_q, len_k = _int32_cuda(seqlens_q, "seqlens_q"), _int32_cuda(seqlens_k, "seqlens_k")
+    packed_q, rows_q, Hq, lay_q = _side_layout(q, "q")
+    packed_k, rows_k, Hkv, lay_k = _side_layout(k, "k")
+    _, _, _, lay_v = _side_layout(v, "v")
+    if packed_q != (cu_q is not None) or packed_k != (cu_k is not None):
+        raise ValueError("a packed (3-D) side needs cu_seqlens; a padded (4-D) side must not have it")
+    if v.shape != k.shape or q.shape[-1] != k.shape[-1]:
+        raise ValueError("q, k, v shapes disagree")
+    D = q.shape[-1]
+    S = cu_q.numel() - 1 if packed_q else q.shape[0]
+    S_k = cu_k.numel() - 1 if packed_k else k.shape[0]
+    if S != S_k or S <= 0:
+        raise ValueError("queries and keys describe different numbers of sequences")
+    if max_seqlen_q is None:  # convenience: one device-to-host read
+        if packed_q:
+            max_seqlen_q = int((cu_q[1:] - cu_q[:-1]).max().item())
+        else:
+            max_seqlen_q = int(len_q.max().item()) if len_q is not None else rows_q
+    max_seqlen_q = max(1, int(max_seqlen_q))
+    if out is None:
+        out = torch.empty_like(q)
+    _, _, _, lay_o = _side_layout(out, "out")
+    lse = None
+    if return_lse:
+        lse = torch.empty(((Hq, rows_q) if packed_q else (S, Hq, rows_q)), dtype=torch.float32,
+                          device=q.device)
+    need = gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = gqa_attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                             _ptr(cu_q), _ptr(cu_k), _ptr(len_q), _ptr(len_k), S, Hq, Hkv, D, rows_q,
+                             rows_k, max_seqlen_q, lay_q, lay_k, lay_v, lay_o, float(scale or 0.0),
+                             int(window), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_fwd_varlen")
+    return (out, lse) if return_lse else out
+
+
+def attn_decode_varlen(q, k_cache, v_cache, seqlens_k, *, block_table=None, max_seqlen_k=None,
+                       pool_layout="NHD", scale=None, window=0, num_splits=0, out=None, workspace=None,
+                       stream=None):
+    """Decode of q [B, Hq, Tq, D] (Tq <= 16; or [B, Hq, D]) over per-sequence cache lengths.
+
+    Contiguous cache (``block_table`` None): k_cache/v_cache [B, Hkv, T_cap, D] with any
+    batch/head/row strides. Paged cache: a pool [pages, page, Hkv, D] ("NHD") or
+    [pages, Hkv, page, D] ("HND") and an int32 block table [B, max_pages]. Sequence b's
+    queries are the last Tq of its seqlens_k[b] positions.
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_bf16_cuda(t, n)
+    seqlens_k = _int32_cuda(seqlens_k, "seqlens_k")
+    table = _int32_cuda(block_table, "block_table")
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    B, Hq, D = q.shape[0], q.shape[1], q.shape[-1]
+    Tq = q.shape[2] if q.dim() == 4 else 1
+    if seqlens_k is None or seqlens_k.numel() != B:
+        raise ValueError("seqlens_k must hold one length per sequence")
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4 or k_cache.stride(3) != 1:
+        raise ValueError("k_cache and v_cache must be 4-D with a contiguous D axis and equal shapes")
+
+    def lay(t):
+        if table is None:
+            return (t.stride(0), t.stride(1), t.stride(2))
+        if pool_layout == "NHD":
+            return (t.stride(0), t.stride(2), t.stride(1))
+        if pool_layout == "HND":
+            return (t.stride(0), t.stride(1), t.stride(2))
+        raise ValueError("pool_layout must be 'NHD' or 'HND'")
+
+    if table is None:
+        Hkv = k_cache.shape[1]
+        page_size = num_pages = max_pages = 0
+        cap = k_cache.shape[2]
+        max_seqlen_k = cap if max_seqlen_k is None else int(max_seqlen_k)
+        if max_seqlen_k > cap:
+            raise ValueError("max_seqlen_k exceeds the cache rows")
+    else:
+        Hkv = k_cache.shape[2] if pool_layout == "NHD" else k_cache.shape[1]
+        page_size = k_cache.shape[1] if pool_layout == "NHD" else k_cache.shape[2]
+        num_pages = k_cache.shape[0]
+        if table.dim() != 2 or table.shape[0] != B:
+            raise ValueError("block_table must be [B, max_pages]")
+        max_pages = table.shape[1]
+        max_seqlen_k = max_pages * page_size if max_seqlen_k is None else int(max_seqlen_k)
+    if out is None:
+        out = torch.empty_like(q)
+    need = gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window, num_splits)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = gqa_attn_decode_varlen(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                seqlens_k.data_ptr(), _ptr(table), page_size, num_pages, max_pages, B, Hq,
+                                Hkv, Tq, max_seqlen_k, D, lay(k_cache), lay(v_cache), float(scale or 0.0),
+                                int(window), int(num_splits), _ptr(workspace),
+                                workspace.numel() if workspace is not None else 0, _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_decode_varlen")
     return out

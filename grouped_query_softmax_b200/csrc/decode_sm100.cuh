@@ -46,6 +46,14 @@ struct DecParams {
     float* ws_lse;           // [splits, B * Hq * Tq] log2-domain log-sum-exp
     uint32_t* err;
     unsigned long long timeout_ns;
+    // ---- per-sequence cache lengths (the kVarlen instantiation only)
+    const int* seqlens;  // [B] cached keys of each sequence (its Tq queries are the last Tq)
+    const int* table;    // [B, max_pages] pool page of each page of a sequence, or null
+    int max_pages;       // block-table row length
+    int page_size;       // keys per page (16, 32, 64 or a multiple of 128)
+    int box_rows;        // rows per TMA box: min(page_size, 128)
+    int num_pages;       // pages in the pool; page coordinates past it read as zeros
+    int capacity;        // most keys a sequence may hold
 };
 
 template <int D>
@@ -74,7 +82,12 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int d) {
     return (uint32_t)(chunk * (kDecKeys * 128) + row * 128 + unit * 16);
 }
 
-template <int D>
+// bf16 pair (keys k, k+1; k in the low half) with the keys at or past `end` zeroed.
+__device__ __forceinline__ uint32_t clear_past(uint32_t pair, int k, int end) {
+    return k >= end ? 0u : (k + 1 >= end ? (pair & 0xFFFFu) : pair);
+}
+
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kDecThreads, 1)
     gqa_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
@@ -97,9 +110,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int g = blockIdx.y / p.n_hc;
     const int hc = blockIdx.y - g * p.n_hc;
     const int b = blockIdx.z;
-    const int blk0 = p.blk_first + split * p.blk_per_split;
-    const int blk1 = min(blk0 + p.blk_per_split, p.n_blk);
-    const int t_end = min(blk1 * kDecKeys, p.Tk);
+    int Tk = p.Tk, blk0, blk1;
+    if constexpr (kVarlen) {
+        // this sequence's own length: its key blocks are shared out over the splits
+        Tk = __ldg(p.seqlens + b);
+        if (Tk < p.Tq || Tk > p.capacity) {  // uniform over the CTA: nothing waits yet
+            if (threadIdx.x == 0) atomicOr(p.err, kDevErrBadSeqlens);
+            return;
+        }
+        const int n_blk = (Tk + kDecKeys - 1) / kDecKeys;
+        const int key_lo = p.window > 0 ? max(0, Tk - p.Tq - p.window + 1) : 0;
+        const int first = key_lo / kDecKeys;
+        const int per = (n_blk - first + p.splits - 1) / p.splits;
+        blk0 = first + split * per;
+        blk1 = min(blk0 + per, n_blk);
+    } else {
+        blk0 = p.blk_first + split * p.blk_per_split;
+        blk1 = min(blk0 + p.blk_per_split, p.n_blk);
+    }
+    const int t_end = min(blk1 * kDecKeys, Tk);
     // Query rows of group g: the G heads' Tq rows each, contiguous in q ((a, i) order).
     const int group_rows = p.G * p.Tq;
     const int rbase = hc * kDecRows;                            // first row of this CTA
@@ -107,8 +136,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const size_t row0 = ((size_t)b * p.Hq + (size_t)g * p.G) * p.Tq + rbase;  // flat row id
     // rows see keys up to their own position (Tk - Tq + i) and, in a window, from
     // position - window + 1; tiles touching either bound are masked element-wise
-    const int pos_min = p.Tk - p.Tq;
-    const int lo_max = p.window > 0 ? p.Tk - p.window : -1;
+    const int pos_min = Tk - p.Tq;
+    const int lo_max = p.window > 0 ? Tk - p.window : -1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -126,7 +155,54 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     float* mrg = reinterpret_cast<float*>(smem);  // merge area, valid after the loop
 
-    if (warp == 0) {
+    if (warp == 0 && kVarlen) {
+        // Whole warp: lanes look up the pool pages of a tile's boxes, lane 0 issues.
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued[kStages];
+        for (int i = 0; i < kStages; ++i) issued[i] = 0;
+        const bool paged = p.table != nullptr;
+        const int n_box = paged ? kDecKeys / p.box_rows : 1;
+        for (int blk = blk0; blk < blk1; ++blk) {
+            int page = b, row = blk * kDecKeys;  // contiguous cache: batch b, rows from blk*128
+            if (paged && lane < n_box) {
+                const int key0 = blk * kDecKeys + lane * p.box_rows;
+                row = key0 % p.page_size;
+                page = key0 < Tk ? __ldg(p.table + (size_t)b * p.max_pages + key0 / p.page_size)
+                                 : p.num_pages;  // past the sequence: an out-of-range page reads zeros
+            }
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag, p.err,
+                                       p.timeout_ns);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            const uint32_t fbar = smem_u32(&ctl->full[stage]);
+            const uint32_t sK = sbase + stage * L::kStageBytes;
+            if (lane == 0) mbar_arrive_expect_tx(fbar, L::kStageBytes);
+            for (int bi = 0; bi < n_box; ++bi) {
+                const int pg = __shfl_sync(0xffffffffu, page, bi);
+                const int rw = __shfl_sync(0xffffffffu, row, bi);
+                if (lane == 0) {
+                    const uint32_t dst = sK + bi * p.box_rows * 128;
+                    for (int c = 0; c < L::kChunks; ++c) {
+                        tma_load_4d(dst + c * L::kChunkBytes, &tm_k, fbar, c * 64, rw, g, pg);
+                        tma_load_4d(dst + L::kTileBytes + c * L::kChunkBytes, &tm_v, fbar, c * 64, rw, g, pg);
+                    }
+                }
+            }
+            ++issued[stage];
+            if (++stage == kStages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (lane == 0 && *abort_flag)
+            for (int i = 0; i < kStages; ++i)
+                if (issued[i])
+                    mbar_wait_drain(smem_u32(&ctl->full[i]), (issued[i] - 1u) & 1u, p.timeout_ns);
+        __syncthreads();  // pairs with the consumers' barrier before the merge
+        __syncthreads();
+    } else if (warp == 0) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -168,7 +244,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int rr = rbase + r_lo + 8 * h;
-            rpos[h] = p.Tk - p.Tq + rr % p.Tq;
+            rpos[h] = Tk - p.Tq + rr % p.Tq;
             rlo[h] = p.window > 0 ? rpos[h] - p.window + 1 : -1;
         }
         {
@@ -261,6 +337,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 }
             }
             // ---- O += P V for this warp's 32 keys
+            // Keys past the sequence's end (rest of a page, padding of a contiguous
+            // cache) hold arbitrary bits; P is 0 there, but 0 * NaN is not, so their
+            // V values are cleared in registers on the sequence's last tile.
+            const bool tail = kVarlen && blk * kDecKeys + kDecKeys > Tk;
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
 #pragma unroll
@@ -270,6 +350,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     const int d = dp * 16 + (mi >> 1) * 8;
                     uint32_t b0, b1, b2, b3;
                     ldmatrix_x4_trans(sV + sw128_off(key, d), b0, b1, b2, b3);
+                    if (tail) {
+                        // this thread holds keys kb, kb+1 (b0, b2) and kb+8, kb+9 (b1, b3),
+                        // the lower key in the low half
+                        const int kb = blk * kDecKeys + cw * 32 + k2 * 16 + c2;
+                        b0 = clear_past(b0, kb, Tk);
+                        b2 = clear_past(b2, kb, Tk);
+                        b1 = clear_past(b1, kb + 8, Tk);
+                        b3 = clear_past(b3, kb + 8, Tk);
+                    }
                     mma_bf16_16816(oacc[dp * 2], pa[k2], b0, b1);
                     mma_bf16_16816(oacc[dp * 2 + 1], pa[k2], b2, b3);
                 }

@@ -67,6 +67,26 @@ struct FwdParams {
     unsigned long long timeout_ns;
 };
 
+// Sequences of different lengths (the kVarlen instantiation only). A kernel parameter
+// of its own: growing FwdParams past ~112 bytes made the dense kernel spill.
+struct FwdVarlenParams {
+    const int* cu_q;  // packed queries: sequence s owns rows cu_q[s] .. cu_q[s+1]-1 (batch 0)
+    const int* cu_k;  // packed keys, likewise
+    const int* len_q; // padded queries (cu_q null): sequence s is batch s, rows 0 .. len_q[s]-1
+    const int* len_k; // padded keys; a null length array means every sequence has all rows
+    int rows_q, rows_k;  // row extent of the q/o and k/v tensors
+    int n_lvl, n_h;      // candidate unit c = (s * n_lvl + level) * n_h + head slot
+    const int* unit_list;   // present units, longest first (written by the plan kernel)
+    const int* unit_count;  // their number
+    long long o_sb, o_sh, o_st;  // element strides of o (batch, head, row); d is contiguous
+};
+
+// Where one sequence's rows are: batch index, first row and length of each side.
+struct SeqGeo {
+    int b_q, r_q, len_q;
+    int b_k, r_k, len_k;
+};
+
 template <int D>
 struct FwdSmem {
     static constexpr int kChunks = D / 64;             // 64-element (128-byte) column chunks
@@ -81,6 +101,7 @@ struct FwdSmem {
         uint64_t q_empty;
         uint64_t full[kStages];
         uint64_t empty[kStages];
+        uint64_t land[kStages];  // ragged last V tile of a sequence: lands here, is cleaned, then full
         uint64_t s_full[2];
         uint64_t p_full[2];
         uint64_t o_full[2];
@@ -100,6 +121,28 @@ struct SubTile {
     int masked_from;  // first KV tile that crosses the causal diagonal
     int lo_masked_end;  // KV tiles below this cross the lower edge of the window
 };
+
+// Key-tile bounds of one sub-tile whose rows sit at positions off + row0 ...
+__device__ __forceinline__ void fwd_fill_subtile(SubTile& st, int len_q, int off, int window) {
+    st.j_begin = 0;
+    st.lo_masked_end = 0;
+    if (st.row0 >= len_q) {
+        st.n_kv = 0;
+        st.masked_from = 0;
+        return;
+    }
+    const int last = min(st.row0 + kFwdRows - 1, len_q - 1);
+    st.n_kv = (off + last) / kFwdKeys + 1;
+    st.masked_from = (off + st.row0 + 1) / kFwdKeys;
+    if (window > 0) {
+        // row positions P0..P1 see keys (P - w, P]: tiles before the first row's
+        // window are skipped, tiles before the last row's window start are masked
+        const int lo_first = off + st.row0 - window + 1;
+        const int lo_last = off + last - window + 1;
+        st.j_begin = lo_first > 0 ? lo_first / kFwdKeys : 0;
+        st.lo_masked_end = lo_last > 0 ? (lo_last + kFwdKeys - 1) / kFwdKeys : 0;
+    }
+}
 
 __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& b, int& g,
                                                 SubTile (&st)[2]) {
@@ -124,26 +167,70 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
         st[1].row0 = st[0].row0 + kFwdRows;
     }
     g = st[0].head / p.G;
+    fwd_fill_subtile(st[0], p.Tq, off, p.window);
+    fwd_fill_subtile(st[1], p.Tq, off, p.window);
+}
+
+// One sequence side: batch index, first row and length.
+__device__ __forceinline__ void fwd_seq_side(const int* cu, const int* len, int rows, int s, int& b,
+                                             int& r, int& l) {
+    if (cu != nullptr) {
+        r = __ldg(cu + s);
+        l = __ldg(cu + s + 1) - r;
+        b = 0;
+    } else {
+        r = 0;
+        l = len != nullptr ? __ldg(len + s) : rows;
+        b = s;
+    }
+}
+
+// Candidate unit c of a variable-length launch: sequence s, row level, head slot.
+__device__ __forceinline__ void fwd_varlen_unit(const FwdParams& p, const FwdVarlenParams& vp, int c,
+                                                SeqGeo& geo, int& g, SubTile (&st)[2]) {
+    const int hidx = c % vp.n_h;
+    const int t = c / vp.n_h;
+    const int lvl = t % vp.n_lvl;
+    const int s = t / vp.n_lvl;
+    fwd_seq_side(vp.cu_q, vp.len_q, vp.rows_q, s, geo.b_q, geo.r_q, geo.len_q);
+    fwd_seq_side(vp.cu_k, vp.len_k, vp.rows_k, s, geo.b_k, geo.r_k, geo.len_k);
+    if (p.pair_heads) {
+        st[0].head = 2 * hidx;
+        st[1].head = 2 * hidx + 1;
+        st[0].row0 = st[1].row0 = lvl * kFwdRows;
+    } else {
+        st[0].head = st[1].head = hidx;
+        st[0].row0 = lvl * 2 * kFwdRows;
+        st[1].row0 = st[0].row0 + kFwdRows;
+    }
+    g = st[0].head / p.G;
+    const int off = geo.len_k - geo.len_q;
+    fwd_fill_subtile(st[0], geo.len_q, off, p.window);
+    fwd_fill_subtile(st[1], geo.len_q, off, p.window);
+}
+
+// KV tiles a unit's sub-tiles visit in total (0 = nothing to compute).
+__device__ __forceinline__ int fwd_unit_work(const SubTile (&st)[2]) {
+    int w = 0;
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-        st[s].j_begin = 0;
-        st[s].lo_masked_end = 0;
-        if (st[s].row0 >= p.Tq) {
-            st[s].n_kv = 0;
-            st[s].masked_from = 0;
-        } else {
-            const int last = min(st[s].row0 + kFwdRows - 1, p.Tq - 1);
-            st[s].n_kv = (off + last) / kFwdKeys + 1;
-            st[s].masked_from = (off + st[s].row0 + 1) / kFwdKeys;
-            if (p.window > 0) {
-                // row positions P0..P1 see keys (P - w, P]: tiles before the first row's
-                // window are skipped, tiles before the last row's window start are masked
-                const int lo_first = off + st[s].row0 - p.window + 1;
-                const int lo_last = off + last - p.window + 1;
-                st[s].j_begin = lo_first > 0 ? lo_first / kFwdKeys : 0;
-                st[s].lo_masked_end = lo_last > 0 ? (lo_last + kFwdKeys - 1) / kFwdKeys : 0;
-            }
-        }
+    for (int s = 0; s < 2; ++s)
+        if (st[s].n_kv > 0) w += st[s].n_kv - st[s].j_begin;
+    return w;
+}
+
+// Unit u of the launch, as the geometry of its sequence and its two sub-tiles.
+template <bool kVarlen>
+__device__ __forceinline__ void fwd_unit(const FwdParams& p, const FwdVarlenParams& vp, int u,
+                                         SeqGeo& geo, int& g, SubTile (&st)[2]) {
+    if constexpr (kVarlen) {
+        fwd_varlen_unit(p, vp, __ldg(vp.unit_list + u), geo, g, st);
+    } else {
+        int b;
+        fwd_decode_unit(p, u, b, g, st);
+        geo.b_q = geo.b_k = b;
+        geo.r_q = geo.r_k = 0;
+        geo.len_q = p.Tq;
+        geo.len_k = p.Tk;
     }
 }
 
@@ -153,11 +240,12 @@ __device__ __forceinline__ int snake_unit(int k, int i, int n) {
     return k * n + ((k & 1) ? (n - 1 - i) : i);
 }
 
-template <int D>
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     gqa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p,
+                         const FwdVarlenParams vp) {
     using L = FwdSmem<D>;
     using Ctl = typename L::Ctl;
     constexpr int kStages = L::kStages;
@@ -180,6 +268,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // longest first, so this striding spreads the causal work evenly over the SMs).
     const int cta = blockIdx.x;
     const int ncta = gridDim.x;
+    // variable-length launches read the unit count the plan kernel wrote
+    const int units = kVarlen ? *reinterpret_cast<const volatile int*>(vp.unit_count) : p.units;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl->q_full), 1);
@@ -187,6 +277,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < kStages; ++i) {
             mbar_init(smem_u32(&ctl->full[i]), 1);
             mbar_init(smem_u32(&ctl->empty[i]), 1);
+            mbar_init(smem_u32(&ctl->land[i]), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&ctl->s_full[s]), 1);
@@ -219,16 +310,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued[kStages];
-            for (int i = 0; i < kStages; ++i) issued[i] = 0;
+            uint32_t landed[kStages];  // copies that completed on land[] (ragged V tiles)
+            bool last_land[kStages];
+            for (int i = 0; i < kStages; ++i) {
+                issued[i] = landed[i] = 0;
+                last_land[i] = false;
+            }
             uint32_t q_loads = 0;
             const uint32_t qbar = smem_u32(&ctl->q_full);
             bool ok = true;
-            for (int k = 0; k * ncta < p.units && ok; ++k) {
+            for (int k = 0; k * ncta < units && ok; ++k) {
                 const int u = snake_unit(k, cta, ncta);
-                if (u >= p.units) continue;
-                int b, g;
+                if (u >= units) continue;
+                int g;
+                SeqGeo geo;
                 SubTile st[2];
-                fwd_decode_unit(p, u, b, g, st);
+                fwd_unit<kVarlen>(p, vp, u, geo, g, st);
                 const int n_max = max(st[0].n_kv, st[1].n_kv);
                 const int jb = st[1].n_kv > 0 ? min(st[0].j_begin, st[1].j_begin) : st[0].j_begin;
                 // the previous unit's Q K^T products must be done before Q is replaced
@@ -240,20 +337,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int s = 0; s < nq; ++s)
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_4d(sQ + s * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64,
-                                    st[s].row0, st[s].head, b);
+                                    geo.r_q + st[s].row0, st[s].head, geo.b_q);
                 ++q_loads;
                 for (int j = jb; j < n_max && ok; ++j) {
                     for (int t = 0; t < 2; ++t) {
                         if (!(ok = mbar_wait_bounded(smem_u32(&ctl->empty[stage]), phase ^ 1u, abort_flag,
                                                      p.err, p.timeout_ns)))
                             break;
-                        const uint32_t fbar = smem_u32(&ctl->full[stage]);
+                        // A V tile that runs past its sequence's last key may hold another
+                        // sequence's rows or padding (even NaN); it lands on land[] and warp 3
+                        // zeroes those rows before it signals full[] (P is 0 there, 0 * NaN is not).
+                        const bool ragged = kVarlen && t == 1 && (j + 1) * kFwdKeys > geo.len_k;
+                        const uint32_t fbar = smem_u32(ragged ? &ctl->land[stage] : &ctl->full[stage]);
                         mbar_arrive_expect_tx(fbar, kTileBytes);
                         const CUtensorMap* map = t ? &tm_v : &tm_k;
                         for (int c = 0; c < L::kChunks; ++c)
                             tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
-                                        j * kFwdKeys, g, b);
+                                        geo.r_k + j * kFwdKeys, g, geo.b_k);
                         ++issued[stage];
+                        if constexpr (kVarlen) {
+                            last_land[stage] = ragged;
+                            if (ragged) ++landed[stage];
+                        }
                         if (++stage == kStages) {
                             stage = 0;
                             phase ^= 1u;
@@ -264,9 +369,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (*abort_flag) {
                 // let every copy this thread started land before the CTA exits
                 if (q_loads) mbar_wait_drain(qbar, (q_loads - 1) & 1u, p.timeout_ns);
-                for (int i = 0; i < kStages; ++i)
-                    if (issued[i])
+                for (int i = 0; i < kStages; ++i) {
+                    if (kVarlen && last_land[i])
+                        mbar_wait_drain(smem_u32(&ctl->land[i]), (landed[i] - 1u) & 1u, p.timeout_ns);
+                    else if (issued[i])
                         mbar_wait_drain(smem_u32(&ctl->full[i]), (issued[i] - 1u) & 1u, p.timeout_ns);
+                }
             }
         }
     } else if (warp == 1) {
@@ -319,12 +427,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                               (accumulate || kk > 0) ? 1u : 0u);
             };
 
-            for (int k = 0; k * ncta < p.units && ok; ++k) {
+            for (int k = 0; k * ncta < units && ok; ++k) {
                 const int u = snake_unit(k, cta, ncta);
-                if (u >= p.units) continue;
-                int b, g;
+                if (u >= units) continue;
+                int g;
+                SeqGeo geo;
                 SubTile st[2];
-                fwd_decode_unit(p, u, b, g, st);
+                fwd_unit<kVarlen>(p, vp, u, geo, g, st);
                 const int n_max = max(st[0].n_kv, st[1].n_kv);
                 // KV tiles jb .. n_max-1; sub-tile s uses tiles st[s].j_begin .. st[s].n_kv-1
                 const int jb = st[1].n_kv > 0 ? min(st[0].j_begin, st[1].j_begin) : st[0].j_begin;
@@ -389,6 +498,55 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_wait_drain(smem_u32(&ctl->drain), 0, p.timeout_ns);
             }
         }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ ragged-tile cleaner
+        // Walks the same units and ring slots as the producer. For each V tile that runs
+        // past its sequence's last key it waits for the copy on land[], zeroes the rows
+        // past that key and releases the slot to the MMA issuer through full[].
+        if constexpr (kVarlen) {
+            int stage = 0;
+            uint32_t land_uses[kStages];
+            for (int i = 0; i < kStages; ++i) land_uses[i] = 0;
+            bool ok = true;
+            for (int k = 0; k * ncta < units && ok; ++k) {
+                const int u = snake_unit(k, cta, ncta);
+                if (u >= units) continue;
+                int g;
+                SeqGeo geo;
+                SubTile st[2];
+                fwd_unit<kVarlen>(p, vp, u, geo, g, st);
+                const int n_max = max(st[0].n_kv, st[1].n_kv);
+                const int jb = st[1].n_kv > 0 ? min(st[0].j_begin, st[1].j_begin) : st[0].j_begin;
+                for (int j = jb; j < n_max && ok; ++j) {
+                    const int vstage = stage + 1 == kStages ? 0 : stage + 1;  // K at stage, V next
+                    if ((j + 1) * kFwdKeys > geo.len_k) {
+                        const uint32_t lbar = smem_u32(&ctl->land[vstage]);
+                        bool got = true;
+                        if (lane == 0)
+                            got = mbar_wait_bounded(lbar, land_uses[vstage] & 1u, abort_flag, p.err,
+                                                    p.timeout_ns);
+                        got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                        ++land_uses[vstage];
+                        if (!got) {
+                            ok = false;
+                            break;
+                        }
+                        // rows keep .. 127 of every 128-byte column chunk (swizzle only
+                        // permutes 16-byte units inside a row, so whole rows are zeroed)
+                        const int keep = geo.len_k - j * kFwdKeys;  // 1 .. 127
+                        const int n16 = (kFwdKeys - keep) * 8;      // 16-byte units per chunk
+                        const uint32_t tile = sRing + vstage * kTileBytes + keep * 128;
+                        for (int c = 0; c < L::kChunks; ++c)
+                            for (int i = lane; i < n16; i += 32)
+                                st_shared_v4(tile + c * kChunkBytes + i * 16, 0u, 0u, 0u, 0u);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&ctl->full[vstage]));
+                    }
+                    stage = vstage + 1 == kStages ? 0 : vstage + 1;
+                }
+            }
+        }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax warpgroups
         setmaxnreg_inc<kFwdSoftmaxRegs>();
@@ -399,17 +557,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t tS = tmem + lane_sel + (uint32_t)(s * 128);
         const uint32_t tO = tmem + lane_sel + 256u + (uint32_t)(s * D);
         const float sl2 = p.scale_log2;
-        const int off = p.Tk - p.Tq;
         uint32_t sph = 0, oph = 0;
         bool ok = true;
-        for (int k = 0; k * ncta < p.units && ok; ++k) {
+        for (int k = 0; k * ncta < units && ok; ++k) {
             const int u = snake_unit(k, cta, ncta);
-            if (u >= p.units) continue;
-            int b, g;
+            if (u >= units) continue;
+            int g;
+            SeqGeo geo;
             SubTile st[2];
-            fwd_decode_unit(p, u, b, g, st);
+            fwd_unit<kVarlen>(p, vp, u, geo, g, st);
             const SubTile me = st[s];
             if (me.n_kv == 0) continue;
+            const int off = geo.len_k - geo.len_q;
             const int pos = off + me.row0 + r;  // absolute position of this query row
             const int lo = pos - p.window + 1;  // first key inside the window (window > 0)
             float m = -INFINITY;  // running max of scaled scores (log2 units)
@@ -543,8 +702,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             oph ^= 1u;
             tc_fence_after_sync();
             const int row = me.row0 + r;
+            const bool row_ok = row < geo.len_q;
             const float inv_l = 1.f / l;
-            __nv_bfloat16* out = p.o + (((size_t)b * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
+            __nv_bfloat16* out;
+            if constexpr (kVarlen)
+                out = p.o + geo.b_q * vp.o_sb + me.head * vp.o_sh + (long long)(geo.r_q + row) * vp.o_st;
+            else
+                out = p.o + (((size_t)geo.b_q * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t orr[32];
@@ -557,7 +721,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int e = 0; e < 16; ++e)
                     pw[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
                                         __uint_as_float(orr[2 * e + 1]) * inv_l);
-                if (row < p.Tq) {
+                if (row_ok) {
                     uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) dst[e] = v4[e];
@@ -566,9 +730,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // O_s has been read: the next unit's first P V may overwrite it
             tc_fence_before_sync();
             mbar_arrive(smem_u32(&ctl->o_empty[s]));
-            if (p.lse != nullptr && row < p.Tq)
-                p.lse[((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row] =
-                    (m + __log2f(l)) * 0.69314718055994530942f;
+            if (p.lse != nullptr && row_ok) {
+                const size_t li = kVarlen ? ((size_t)geo.b_q * p.Hq + me.head) * (size_t)vp.rows_q + geo.r_q + row
+                                          : ((size_t)geo.b_q * p.Hq + me.head) * (size_t)p.Tq + row;
+                p.lse[li] = (m + __log2f(l)) * 0.69314718055994530942f;
+            }
         }
     }
 
@@ -578,6 +744,102 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
+}
+
+
+// ---------------------------------------------------------------- variable-length plan
+// One CTA. Checks every sequence's bounds against the tensors, then lists the units
+// that have work, ordered by decreasing KV-tile count (a counting sort over buckets),
+// so the persistent kernel's boustrophedon walk keeps its balance when sequences
+// differ in length. Workspace: ws[0] = unit count, units from ws[kPlanHeaderInts].
+// A sequence outside its tensor (or with more queries than keys) sets
+// kDevErrBadSeqlens and an empty list: nothing is computed, nothing is written.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 4 * kPlanThreads;
+constexpr int kPlanHeaderInts = 64;  // 256 bytes
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+    gqa_fwd_varlen_plan_kernel(const FwdParams p, const FwdVarlenParams vp, int S, int max_q,
+                               long long n_cand, int* ws) {
+    __shared__ int hist[kPlanBuckets];
+    __shared__ int warp_sum[32];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    for (int i = tid; i < kPlanBuckets; i += kPlanThreads) hist[i] = 0;
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    for (int s = tid; s < S; s += kPlanThreads) {
+        int bq, rq, lq, bk, rk, lk;
+        fwd_seq_side(vp.cu_q, vp.len_q, vp.rows_q, s, bq, rq, lq);
+        fwd_seq_side(vp.cu_k, vp.len_k, vp.rows_k, s, bk, rk, lk);
+        const bool ok = rq >= 0 && lq >= 0 && (long long)rq + lq <= vp.rows_q && rk >= 0 && lk >= 0 &&
+                        (long long)rk + lk <= vp.rows_k && lq <= lk && lq <= max_q;
+        if (!ok) bad = 1;
+    }
+    __syncthreads();
+    if (bad) {
+        if (tid == 0) {
+            ws[0] = 0;
+            atomicOr(p.err, kDevErrBadSeqlens);
+        }
+        return;
+    }
+    for (long long c = tid; c < n_cand; c += kPlanThreads) {
+        SeqGeo geo;
+        int g;
+        SubTile st[2];
+        fwd_varlen_unit(p, vp, (int)c, geo, g, st);
+        const int w = fwd_unit_work(st);
+        if (w > 0) atomicAdd(&hist[min(w, kPlanBuckets - 1)], 1);
+    }
+    __syncthreads();
+    // bucket b starts after every unit in buckets above it: thread t owns buckets
+    // 4t .. 4t+3; an ascending block scan of the per-thread totals gives the rest
+    int cnt[4], mine = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        cnt[e] = hist[4 * tid + e];
+        mine += cnt[e];
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int x = warp_sum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        warp_sum[lane] = x;
+    }
+    __syncthreads();
+    incl += warp > 0 ? warp_sum[warp - 1] : 0;
+    const int total = warp_sum[31];
+    int cursor = total - incl;  // units in buckets owned by higher threads
+#pragma unroll
+    for (int e = 3; e >= 0; --e) {
+        hist[4 * tid + e] = cursor;
+        cursor += cnt[e];
+    }
+    __syncthreads();
+    int* list = ws + kPlanHeaderInts;
+    for (long long c = tid; c < n_cand; c += kPlanThreads) {
+        SeqGeo geo;
+        int g;
+        SubTile st[2];
+        fwd_varlen_unit(p, vp, (int)c, geo, g, st);
+        const int w = fwd_unit_work(st);
+        if (w > 0) list[atomicAdd(&hist[min(w, kPlanBuckets - 1)], 1)] = (int)c;
+    }
+    if (tid == 0) ws[0] = total;
 }
 
 }  // namespace gqa

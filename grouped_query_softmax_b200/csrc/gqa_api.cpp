@@ -35,15 +35,16 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// A [B, H, T, D] bf16 view with packed rows and free (b, h) strides, tiled as boxes of
-// 128 rows x 64 columns (128 bytes) with the 128-byte swizzle. Strides in elements.
+// A [B, H, T, D] bf16 view with free (b, h, t) strides (d contiguous), tiled as boxes of
+// box_rows rows x 64 columns (128 bytes) with the 128-byte swizzle. Strides in elements.
 gqa_status make_map(CUtensorMap* map, const void* base, int B, int H, int T, int D,
-                    long long s_b, long long s_h) {
+                    long long s_b, long long s_h, long long s_t = -1, int box_rows = gqa::kTileRows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return GQA_ERR_CUDA;
+    if (s_t < 0) s_t = D;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)s_h * 2, (cuuint64_t)s_b * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)gqa::kTileRows, 1, 1};
+    cuuint64_t strides[3] = {(cuuint64_t)s_t * 2, (cuuint64_t)s_h * 2, (cuuint64_t)s_b * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -63,6 +64,21 @@ gqa_status check_kv_strides(int B, int Hkv, int Tk, int D, long long& sb, long l
     if (sb <= 0 || sh <= 0) return GQA_ERR_INVALID_ARGUMENT;
     if ((sb & 7) || (sh & 7)) return GQA_ERR_INVALID_ARGUMENT;  // 16-byte TMA strides
     if (sb * 2 >= (1LL << 40) || sh * 2 >= (1LL << 40)) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+// Strides of a gqa_layout over extents (B, H, rows): used ones must be positive
+// multiples of 8 elements (16-byte TMA strides), rows at least D apart; unused ones
+// (extent 1) get a harmless legal value.
+gqa_status check_layout(const gqa_layout* l, int B, int H, int rows, int D, long long& sb,
+                        long long& sh, long long& st) {
+    if (l == nullptr) return GQA_ERR_INVALID_ARGUMENT;
+    st = effective_stride(l->st, rows, D);
+    sh = effective_stride(l->sh, H, st * rows);
+    sb = effective_stride(l->sb, B, sh * H);
+    if (st < D || sh <= 0 || sb <= 0) return GQA_ERR_INVALID_ARGUMENT;
+    if ((st & 7) || (sh & 7) || (sb & 7)) return GQA_ERR_INVALID_ARGUMENT;
+    if (st * 2 >= (1LL << 40) || sh * 2 >= (1LL << 40) || sb * 2 >= (1LL << 40)) return GQA_ERR_UNSUPPORTED;
     return GQA_OK;
 }
 
@@ -243,11 +259,123 @@ gqa_status gqa_attn_decode(const void* q, const void* k_cache, const void* v_cac
                               softmax_scale, 0, num_splits, workspace, workspace_bytes, stream);
 }
 
+size_t gqa_attn_fwd_varlen_workspace_bytes(int S, int Hq, int Hkv, int max_seqlen_q) {
+    if (S <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seqlen_q <= 0) return 0;
+    int n_lvl = 0, n_h = 0;
+    const long long n = gqa::fwd_varlen_candidates(S, Hq, Hkv, max_seqlen_q, &n_lvl, &n_h);
+    if (n <= 0 || n > 0x7fffffffLL - 64) return 0;
+    return gqa::fwd_varlen_workspace_bytes(n);
+}
+
+gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqlens_q,
+                               const int* seqlens_k, int S, int Hq, int Hkv, int D, int rows_q,
+                               int rows_k, int max_seqlen_q, const gqa_layout* q_layout,
+                               const gqa_layout* k_layout, const gqa_layout* v_layout,
+                               const gqa_layout* o_layout, float softmax_scale, int window,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    if (S <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || rows_q <= 0 || rows_k <= 0 || max_seqlen_q <= 0)
+        return GQA_ERR_INVALID_ARGUMENT;
+    if (Hq % Hkv != 0 || window < 0) return GQA_ERR_INVALID_ARGUMENT;
+    if (D != 64 && D != 128) return GQA_ERR_UNSUPPORTED;
+    if ((cu_seqlens_q && seqlens_q) || (cu_seqlens_k && seqlens_k)) return GQA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GQA_ERR_INVALID_ARGUMENT;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    const int bq = cu_seqlens_q ? 1 : S;  // batch extent of each side
+    const int bk = cu_seqlens_k ? 1 : S;
+    gqa::FwdVarlenLaunch a{};
+    long long ls[3][3];  // (sb, sh, st) of q, k, v
+    gqa_status e;
+    if ((e = check_layout(q_layout, bq, Hq, rows_q, D, ls[0][0], ls[0][1], ls[0][2])) != GQA_OK) return e;
+    if ((e = check_layout(k_layout, bk, Hkv, rows_k, D, ls[1][0], ls[1][1], ls[1][2])) != GQA_OK) return e;
+    if ((e = check_layout(v_layout, bk, Hkv, rows_k, D, ls[2][0], ls[2][1], ls[2][2])) != GQA_OK) return e;
+    if ((e = check_layout(o_layout, bq, Hq, rows_q, D, a.o_sb, a.o_sh, a.o_st)) != GQA_OK) return e;
+    const size_t need = gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q);
+    if (need == 0) return GQA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GQA_ERR_WORKSPACE;
+    if ((e = make_map(&a.tm_q, q, bq, Hq, rows_q, D, ls[0][0], ls[0][1], ls[0][2])) != GQA_OK) return e;
+    if ((e = make_map(&a.tm_k, k, bk, Hkv, rows_k, D, ls[1][0], ls[1][1], ls[1][2])) != GQA_OK) return e;
+    if ((e = make_map(&a.tm_v, v, bk, Hkv, rows_k, D, ls[2][0], ls[2][1], ls[2][2])) != GQA_OK) return e;
+    a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D;
+    a.rows_q = rows_q; a.rows_k = rows_k; a.max_q = max_seqlen_q;
+    a.window = window;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.cu_q = cu_seqlens_q; a.cu_k = cu_seqlens_k;
+    a.len_q = seqlens_q; a.len_k = seqlens_k;
+    a.o = o;
+    a.lse = lse;
+    a.ws = static_cast<int*>(workspace);
+    return gqa::launch_fwd_varlen(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                  const int* seqlens_k, const int* block_table, int page_size,
+                                  int num_pages, int max_pages, int B, int Hq, int Hkv, int Tq,
+                                  int max_seqlen_k, int D, const gqa_layout* k_layout,
+                                  const gqa_layout* v_layout, float softmax_scale, int window,
+                                  int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+    gqa_status st = check_decode(B, Hq, Hkv, Tq, max_seqlen_k, D, window);
+    if (st != GQA_OK) return st;
+    if (!seqlens_k) return GQA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+        return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    gqa::DecLaunch a{};
+    long long lk[3], lv[3];  // (sb, sh, st)
+    int capacity = max_seqlen_k, box = gqa::kTileKeys;
+    const int b_ext = block_table ? num_pages : B, rows_ext = block_table ? page_size : max_seqlen_k;
+    if (block_table) {
+        const bool page_ok = page_size >= 16 && page_size % 16 == 0 &&
+                             (page_size % gqa::kTileKeys == 0 || gqa::kTileKeys % page_size == 0);
+        if (!page_ok || num_pages <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARGUMENT;
+        box = page_size < gqa::kTileKeys ? page_size : gqa::kTileKeys;
+        capacity = (long long)max_pages * page_size < max_seqlen_k ? max_pages * page_size : max_seqlen_k;
+    } else {
+        page_size = num_pages = max_pages = 0;
+    }
+    if ((st = check_layout(k_layout, b_ext, Hkv, rows_ext, D, lk[0], lk[1], lk[2])) != GQA_OK) return st;
+    if ((st = check_layout(v_layout, b_ext, Hkv, rows_ext, D, lv[0], lv[1], lv[2])) != GQA_OK) return st;
+    // The split count is planned for the longest sequence; each sequence shares its
+    // own blocks over those splits on the device.
+    const SplitPlan sp = plan_splits(B, Hq, Hkv, Tq, max_seqlen_k, window >= max_seqlen_k ? 0 : window,
+                                     num_splits);
+    const long long rows = (long long)B * Hq * Tq;
+    if (sp.splits > 1) {
+        const size_t need = ws_bytes_for(sp, rows, D);
+        if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return GQA_ERR_WORKSPACE;
+        a.ws_o = static_cast<float*>(workspace);
+        a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_lse_offset(sp.splits, rows, D));
+    }
+    if ((st = make_map(&a.tm_k, k_cache, b_ext, Hkv, rows_ext, D, lk[0], lk[1], lk[2], box)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_v, v_cache, b_ext, Hkv, rows_ext, D, lv[0], lv[1], lv[2], box)) != GQA_OK) return st;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = max_seqlen_k; a.D = D;
+    a.window = window;
+    a.splits = sp.splits;
+    a.blk_per_split = sp.blk_per_split;
+    a.blk_first = sp.blk_first;
+    a.n_blk = sp.n_blk;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.q = q;
+    a.o = o;
+    a.seqlens = seqlens_k;
+    a.table = block_table;
+    a.max_pages = max_pages;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.capacity = capacity;
+    return gqa::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 gqa_status gqa_get_device_error(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
     uint32_t v = 0;
     if (gqa::read_and_clear_device_error(&v) != cudaSuccess) return GQA_ERR_CUDA;
-    return v ? GQA_ERR_TIMEOUT : GQA_OK;
+    if (v & 1u) return GQA_ERR_TIMEOUT;  // a bounded wait ran out
+    if (v & 2u) return GQA_ERR_INVALID_ARGUMENT;  // sequence bounds outside their tensors
+    return GQA_OK;
 }
 
 gqa_status gqa_selftest_bounded_wait(unsigned long long timeout_ns, void* stream) {

@@ -17,6 +17,40 @@ struct FwdLaunch {
     float* lse;
 };
 
+// Sequences of different lengths (gqa_attn_fwd_varlen). Exactly one of cu_* / len_*
+// describes each side (both null: every sequence owns all rows of its batch).
+struct FwdVarlenLaunch {
+    CUtensorMap tm_q, tm_k, tm_v;
+    int S, Hq, Hkv, D;
+    int rows_q, rows_k, max_q;
+    int window;
+    float scale;
+    const int* cu_q;
+    const int* cu_k;
+    const int* len_q;
+    const int* len_k;
+    void* o;
+    long long o_sb, o_sh, o_st;  // elements
+    float* lse;
+    int* ws;  // plan workspace (fwd_varlen_workspace_bytes)
+};
+
+// Candidate units of a variable-length forward: S x row levels x head slots. A unit
+// is a head pair (even group size) or a pair of 128-row tiles of one head.
+inline long long fwd_varlen_candidates(int S, int Hq, int Hkv, int max_q, int* n_lvl, int* n_h) {
+    const int G = Hq / Hkv;
+    const bool pair_heads = G % 2 == 0;
+    const int n_qt = (max_q + 127) / 128;
+    *n_lvl = pair_heads ? n_qt : (n_qt + 1) / 2;
+    *n_h = pair_heads ? Hq / 2 : Hq;
+    return (long long)S * *n_lvl * *n_h;
+}
+
+constexpr size_t kPlanHeaderBytes = 256;
+inline size_t fwd_varlen_workspace_bytes(long long candidates) {
+    return kPlanHeaderBytes + (size_t)candidates * sizeof(int);
+}
+
 struct DecLaunch {
     CUtensorMap tm_k, tm_v;
     int B, Hq, Hkv, Tq, Tk, D;
@@ -27,10 +61,15 @@ struct DecLaunch {
     void* o;
     float* ws_o;
     float* ws_lse;
+    // per-sequence lengths (gqa_attn_decode_varlen); seqlens null = the dense path
+    const int* seqlens;
+    const int* table;
+    int max_pages, page_size, num_pages, capacity;
 };
 
 // Each returns cudaSuccess or the launch error; nothing is synchronised.
 cudaError_t launch_fwd(const FwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_fwd_varlen(const FwdVarlenLaunch& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream);
 cudaError_t launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream);
 

@@ -54,17 +54,18 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const int smem = FwdSmem<D>::kBytes;
-    e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // The in-kernel register split (setmaxnreg) needs exactly the launch allocation it
     // was sized for; never launch a build where that does not hold.
     cudaFuncAttributes fa{};
-    e = cudaFuncGetAttributes(&fa, gqa_fwd_sm100_kernel<D>);
+    e = cudaFuncGetAttributes(&fa, gqa_fwd_sm100_kernel<D, false>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
     // persistent: one CTA per SM (shared memory and TMEM allow exactly one)
     const unsigned grid = (unsigned)std::min<long long>(units, sms > 0 ? sms : 1);
-    gqa_fwd_sm100_kernel<D><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    gqa_fwd_sm100_kernel<D, false><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p,
+                                                                         FwdVarlenParams{});
     return cudaGetLastError();
 }
 
@@ -73,6 +74,61 @@ cudaError_t launch_fwd(const FwdLaunch& a, cudaStream_t stream) {
 }
 
 template <int D>
+static cudaError_t launch_fwd_varlen_d(const FwdVarlenLaunch& a, cudaStream_t stream) {
+    FwdParams p{};
+    p.B = a.S;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.G = a.Hq / a.Hkv;
+    p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+    FwdVarlenParams vp{};
+    const long long n_cand = fwd_varlen_candidates(a.S, a.Hq, a.Hkv, a.max_q, &vp.n_lvl, &vp.n_h);
+    if (n_cand <= 0 || n_cand > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.window = a.window;
+    p.o = static_cast<__nv_bfloat16*>(a.o);
+    p.lse = a.lse;
+    p.err = device_error_ptr();
+    p.timeout_ns = kWaitTimeoutNs;
+    if (!p.err) return cudaErrorUnknown;
+    vp.cu_q = a.cu_q;
+    vp.cu_k = a.cu_k;
+    vp.len_q = a.len_q;
+    vp.len_k = a.len_k;
+    vp.rows_q = a.rows_q;
+    vp.rows_k = a.rows_k;
+    vp.unit_count = a.ws;
+    vp.unit_list = a.ws + kPlanHeaderInts;
+    vp.o_sb = a.o_sb;
+    vp.o_sh = a.o_sh;
+    vp.o_st = a.o_st;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int smem = FwdSmem<D>::kBytes;
+    e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, gqa_fwd_sm100_kernel<D, true>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
+    gqa_fwd_varlen_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, vp, a.S, a.max_q, n_cand, a.ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)std::min<long long>(n_cand, sms > 0 ? sms : 1);
+    gqa_fwd_sm100_kernel<D, true><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p, vp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_varlen(const FwdVarlenLaunch& a, cudaStream_t stream) {
+    return a.D == 128 ? launch_fwd_varlen_d<128>(a, stream) : launch_fwd_varlen_d<64>(a, stream);
+}
+
+static_assert(kPlanHeaderInts * sizeof(int) == kPlanHeaderBytes, "plan workspace header");
+
+template <int D, bool kVarlen>
 static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
     DecParams p{};
     p.B = a.B;
@@ -95,12 +151,19 @@ static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
     p.err = device_error_ptr();
     p.timeout_ns = kWaitTimeoutNs;
     if (!p.err) return cudaErrorUnknown;
+    p.seqlens = a.seqlens;
+    p.table = a.table;
+    p.max_pages = a.max_pages;
+    p.page_size = a.page_size;
+    p.box_rows = a.page_size > 0 && a.page_size < kDecKeys ? a.page_size : kDecKeys;
+    p.num_pages = a.num_pages;
+    p.capacity = a.capacity;
     const int smem = DecSmem<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(gqa_decode_sm100_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(gqa_decode_sm100_kernel<D, kVarlen>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.splits, (unsigned)(a.Hkv * p.n_hc), (unsigned)a.B);
-    gqa_decode_sm100_kernel<D><<<grid, kDecThreads, smem, stream>>>(a.tm_k, a.tm_v, p);
+    gqa_decode_sm100_kernel<D, kVarlen><<<grid, kDecThreads, smem, stream>>>(a.tm_k, a.tm_v, p);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
     const int rows = a.B * a.Hq * a.Tq;
@@ -110,7 +173,9 @@ static cudaError_t launch_decode_d(const DecLaunch& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream) {
-    return a.D == 128 ? launch_decode_d<128>(a, stream) : launch_decode_d<64>(a, stream);
+    if (a.seqlens != nullptr)
+        return a.D == 128 ? launch_decode_d<128, true>(a, stream) : launch_decode_d<64, true>(a, stream);
+    return a.D == 128 ? launch_decode_d<128, false>(a, stream) : launch_decode_d<64, false>(a, stream);
 }
 
 // One CTA, one thread: wait on an mbarrier that never completes, bounded by

@@ -14,6 +14,7 @@ namespace gqa {
 // gqa_get_device_error(). Defined once in gqa_kernels.cu.
 enum : uint32_t {
     kDevErrWaitTimeout = 1u,  // a bounded mbarrier wait ran out
+    kDevErrBadSeqlens = 2u,   // sequence lengths / boundaries outside the tensors (nothing computed)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

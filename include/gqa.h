@@ -31,7 +31,9 @@
  * Errors: argument checks run on the host before anything is enqueued; a call that
  * returns an error has launched nothing. Launch failures return GQA_ERR_CUDA.
  * Device-side waits are bounded; a wait that runs out sets a device error word
- * that gqa_get_device_error() reports as GQA_ERR_TIMEOUT.
+ * that gqa_get_device_error() reports as GQA_ERR_TIMEOUT. Sequence bounds that
+ * live on the device (the *_varlen calls) are checked there and reported the same
+ * way, as GQA_ERR_INVALID_ARGUMENT.
  */
 #ifndef GQA_H_
 #define GQA_H_
@@ -167,14 +169,112 @@ GQA_API gqa_status gqa_attn_decode_ex(const void* q, const void* k_cache, const 
 /* The split count gqa_attn_decode will use for these arguments (num_splits 0 = auto). */
 GQA_API int gqa_attn_decode_num_splits(int B, int Hq, int Hkv, int Tk, int D, int num_splits);
 
+/*
+ * Element strides of one bf16 operand: element (b, h, t, d) is at
+ * base + b*sb + h*sh + t*st + d (elements; d is contiguous). Every stride used must
+ * be a positive multiple of 8 elements (16 bytes, a TMA requirement) and st >= D.
+ * A stride along an axis of extent 1 is not used.
+ *   head-major  [H, rows, D]:     sh = rows*D, st = D
+ *   token-major [rows, H, D]:     sh = D,      st = H*D   (serving engines' packed layout)
+ *   padded      [B, H, rows, D]:  sb = H*rows*D, sh = rows*D, st = D
+ *   paged pool  [pages, page, H, D]: sb = page*H*D, sh = D, st = H*D (b = pool page)
+ */
+typedef struct gqa_layout {
+    long long sb, sh, st;
+} gqa_layout;
+
+/*
+ * Sequences of different lengths: S independent causal problems in one call. The
+ * pages ask an attention implementation for padding masks and packed segments, for
+ * query lengths that differ from the cache length, and for masks built from each
+ * sequence's own positions, not from the tensors' shapes ("注意力家族", section
+ * Mask 与增量位置); "Attention Architecture Evolution", section GDN, names the packed
+ * boundaries cu_seqlens. Sequence s has L_q(s) query rows at positions
+ * L_k(s) - L_q(s) .. L_k(s) - 1 of its own L_k(s) keys; no row sees another sequence's
+ * keys or any padding.
+ *
+ * Each side, queries (q, o, lse) and keys (k, v), is either
+ *   packed  cu_seqlens_x non-NULL: int32 [S + 1] on the device, non-decreasing;
+ *           sequence s owns rows cu[s] .. cu[s+1]-1 of a tensor with rows_x rows and
+ *           no batch axis; or
+ *   padded  cu_seqlens_x NULL: sequence s is batch s of an [S, H, rows_x, D] tensor
+ *           and owns its rows 0 .. seqlens_x[s]-1 (seqlens_x int32 [S] on the device;
+ *           NULL = all rows_x rows).
+ * Giving both cu_seqlens_x and seqlens_x for one side is GQA_ERR_INVALID_ARGUMENT.
+ *
+ *   q, k, v, o    bf16 device pointers, 16-byte aligned, addressed through the
+ *                 layouts (see gqa_layout); o is written on the rows of sequences
+ *                 only and must not overlap the inputs.
+ *   lse           fp32 or NULL: the natural-log log-sum-exp of row t of head h of
+ *                 batch b at lse[(b*Hq + h)*rows_q + t] (b = 0 for packed queries).
+ *   max_seqlen_q  >= every L_q(s); sizes the work decomposition and the workspace.
+ *   window        0 = causal; > 0 = sliding window, as for gqa_attn_fwd_ex.
+ *   workspace     device, >= gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv,
+ *                 max_seqlen_q) bytes, 256-byte aligned; contents on entry ignored;
+ *                 not shared by calls that can overlap on the GPU.
+ * Sequence bounds live on the device and are checked there (no host sync): if any
+ * sequence reaches past its tensor's rows or has L_q > L_k or L_q > max_seqlen_q,
+ * the call computes and writes nothing, and the next gqa_get_device_error()
+ * returns GQA_ERR_INVALID_ARGUMENT. Empty sequences (L_q = 0) are allowed.
+ * Work: a small planning kernel lists the (sequence, rows, heads) units that have
+ * work, longest first; the attention kernel then runs over that list.
+ */
+GQA_API size_t gqa_attn_fwd_varlen_workspace_bytes(int S, int Hq, int Hkv, int max_seqlen_q);
+GQA_API gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                       float* lse, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                       const int* seqlens_q, const int* seqlens_k, int S, int Hq,
+                                       int Hkv, int D, int rows_q, int rows_k, int max_seqlen_q,
+                                       const gqa_layout* q_layout, const gqa_layout* k_layout,
+                                       const gqa_layout* v_layout, const gqa_layout* o_layout,
+                                       float softmax_scale, int window, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
+ * Decode over a cache whose sequences have different lengths, contiguous or paged.
+ * Sequence b holds L(b) = seqlens_k[b] keys; its T_q new queries are the last T_q of
+ * them (positions L(b) - T_q .. L(b) - 1), as for gqa_attn_decode_ex. Each sequence's
+ * key blocks are shared out over the splits, so short sequences are not charged for
+ * the longest one's blocks.
+ *
+ *   q, o        bf16 [B, Hq, Tq, D], contiguous; 1 <= Tq <= 16.
+ *   seqlens_k   int32 [B] on the device.
+ *   block_table NULL: contiguous cache; k/v element (b, h, t, d) at the layout's
+ *               b*sb + h*sh + t*st + d, rows 0 .. max_seqlen_k-1 of each sequence.
+ *               Non-NULL: paged cache; int32 [B, max_pages] on the device. Position t
+ *               of sequence b is row t % page_size of pool page
+ *               block_table[b*max_pages + t/page_size]; pool element (page, h, r, d)
+ *               at page*sb + h*sh + r*st + d, num_pages pages. page_size must be 16,
+ *               32, 64 or a multiple of 128. Table entries past a sequence's last page
+ *               are never read; a page number outside [0, num_pages) reads zeros.
+ *   max_seqlen_k  >= every L(b); sizes the split plan (and, for a contiguous cache,
+ *               the rows the cache must hold).
+ *   window, num_splits, workspace   as for gqa_attn_decode_ex; the workspace size is
+ *               gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D,
+ *               window, num_splits).
+ * Every L(b) must lie in [Tq, capacity], capacity = max_seqlen_k for a contiguous
+ * cache and min(max_seqlen_k, max_pages*page_size) for a paged one. It is checked on
+ * the device: a sequence outside that range gets no output and the next
+ * gqa_get_device_error() returns GQA_ERR_INVALID_ARGUMENT. Keys past L(b) (the rest
+ * of a page, a contiguous cache's unused rows) may hold any bits, NaN included.
+ */
+GQA_API gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void* v_cache,
+                                          void* o, const int* seqlens_k, const int* block_table,
+                                          int page_size, int num_pages, int max_pages, int B, int Hq,
+                                          int Hkv, int Tq, int max_seqlen_k, int D,
+                                          const gqa_layout* k_layout, const gqa_layout* v_layout,
+                                          float softmax_scale, int window, int num_splits,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* A static, human-readable name for a status code. */
 GQA_API const char* gqa_status_string(gqa_status s);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device. Returns GQA_ERR_TIMEOUT if a bounded wait in any kernel of this
- * library ran out since the last call, GQA_ERR_CUDA if the stream reports a CUDA
- * error, else GQA_OK.
+ * library ran out since the last call, else GQA_ERR_INVALID_ARGUMENT if a
+ * variable-length call found sequence bounds outside its tensors (see
+ * gqa_attn_fwd_varlen, gqa_attn_decode_varlen), GQA_ERR_CUDA if the stream reports
+ * a CUDA error, else GQA_OK.
  */
 GQA_API gqa_status gqa_get_device_error(void* stream);
 

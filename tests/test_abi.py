@@ -112,3 +112,60 @@ def test_product_does_not_reference_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".cpp", ".h")):
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "gqa_oracle" not in txt, f
+
+
+def varlen_fwd(gqa, **kw):
+    rows = 64
+    lay = (0, 64, 4 * 64)  # token-major [rows, 4, 64]
+    lay_k = (0, 64, 2 * 64)
+    a = dict(q=P, k=P, v=P, o=P, lse=None, cu_seqlens_q=P, cu_seqlens_k=P, seqlens_q=None,
+             seqlens_k=None, S=2, Hq=4, Hkv=2, D=64, rows_q=rows, rows_k=rows, max_seqlen_q=40,
+             q_layout=lay, k_layout=lay_k, v_layout=lay_k, o_layout=lay, softmax_scale=0.0, window=0,
+             workspace=P, workspace_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_fwd_varlen(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(k=P + 8), 1), (dict(lse=P + 2), 1),
+    (dict(S=0), 1), (dict(Hq=3), 1), (dict(rows_q=0), 1), (dict(max_seqlen_q=0), 1),
+    (dict(D=96), 2), (dict(window=-1), 1),
+    (dict(seqlens_q=P), 1),                                   # packed and padded on one side
+    (dict(q_layout=(0, 64, 100)), 1),                         # row stride not a multiple of 8
+    (dict(k_layout=(0, 64, 32)), 1),                          # rows closer than D
+    (dict(o_layout=(0, 0, 256)), 1),                          # zero head stride with 4 heads
+    (dict(cu_seqlens_q=None, q_layout=(0, 64, 256)), 1),      # padded, 2 batches, zero batch stride
+    (dict(workspace=None), 3), (dict(workspace_bytes=64), 3), (dict(workspace=P + 16), 3),
+])
+def test_varlen_fwd_rejects_bad_arguments(gqa, kw, status):
+    assert varlen_fwd(gqa, **kw) == status
+
+
+def test_varlen_workspace_sizes(gqa):
+    # 4 heads over 2 KV heads (G = 2, head pairs): S * ceil(max_q/128) * Hq/2 units + a header
+    assert gqa.gqa_attn_fwd_varlen_workspace_bytes(2, 4, 2, 300) == 256 + 4 * 2 * 3 * 2
+    # G = 3 (row pairs): S * ceil(ceil(max_q/128)/2) * Hq
+    assert gqa.gqa_attn_fwd_varlen_workspace_bytes(2, 6, 2, 300) == 256 + 4 * 2 * 2 * 6
+    assert gqa.gqa_attn_fwd_varlen_workspace_bytes(0, 4, 2, 300) == 0
+    assert gqa.gqa_attn_fwd_varlen_workspace_bytes(2, 5, 2, 300) == 0
+
+
+def varlen_dec(gqa, **kw):
+    a = dict(q=P, k_cache=P, v_cache=P, o=P, seqlens_k=P, block_table=P, page_size=64, num_pages=100,
+             max_pages=16, B=2, Hq=4, Hkv=2, Tq=1, max_seqlen_k=1024, D=128,
+             k_layout=(64 * 2 * 128, 128, 2 * 128), v_layout=(64 * 2 * 128, 128, 2 * 128),
+             softmax_scale=0.0, window=0, num_splits=1, workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_decode_varlen(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(seqlens_k=None), 1), (dict(q=None), 1), (dict(Tq=17), 2), (dict(D=96), 2),
+    (dict(page_size=48), 1), (dict(page_size=8), 1), (dict(page_size=200), 1),
+    (dict(num_pages=0), 1), (dict(max_pages=0), 1),
+    (dict(k_layout=(64 * 2 * 128, 128, 100)), 1),
+    (dict(num_splits=4), 3),                                  # splits need a workspace
+    (dict(block_table=None, k_layout=(0, 1024 * 128, 128)), 1),  # contiguous: 2 sequences, no batch stride
+])
+def test_varlen_decode_rejects_bad_arguments(gqa, kw, status):
+    assert varlen_dec(gqa, **kw) == status
