@@ -286,6 +286,73 @@ def measure_decode(w, steps, warmup, world, dev, e2e_steps):
     return res
 
 
+def varlen_flops(w) -> float:
+    """4 * D * Hq * sum over sequences of their causal-visible pairs."""
+    lq, lk = w.lengths()
+    return 4.0 * w.D * w.Hq * sum(visible_pairs(int(a), int(b), w.window) for a, b in zip(lq, lk) if a)
+
+
+def paged_kv_bytes(w) -> int:
+    """K + V bytes of every cached key, read once per KV head."""
+    return 2 * int(w.lengths().sum()) * w.Hkv * w.D * 2
+
+
+def measure_varlen(w, steps, warmup, world, dev):
+    """gqa_attn_fwd_varlen on a packed workload (plan kernel + attention kernel per step)."""
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, k, v, cu_q, cu_k = w.make()
+    lq, _ = w.lengths()
+    qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
+    cq = torch.tensor(cu_q, device=dev)
+    ck = torch.tensor(cu_k, device=dev)
+    od = torch.empty_like(qd)
+    max_q = int(lq.max())
+    ws = torch.empty(gqa.gqa_attn_fwd_varlen_workspace_bytes(w.S, w.Hq, w.Hkv, max_q), dtype=torch.uint8,
+                     device=dev)
+    fn = lambda: gqa.attn_fwd_varlen(qd, kd, vd, cu_seqlens_q=cq, cu_seqlens_k=ck, max_seqlen_q=max_q,
+                                     window=w.window, out=od, workspace=ws)
+    ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after varlen timing: {gqa.gqa_status_string(st)}")
+    del qd, kd, vd, od, ws
+    torch.cuda.empty_cache()
+    return {"ms_total": ms, "launches": 2 * steps, "tokens_q": int(cu_q[-1]), "tokens_k": int(cu_k[-1])}
+
+
+def measure_paged_decode(w, steps, warmup, world, dev):
+    """gqa_attn_decode_varlen over the paged pool of a PagedDecodeWorkload."""
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, kp, vp, lens, table = w.make()
+    qd, kd, vd = to_device(q, dev), to_device(kp, dev), to_device(vp, dev)
+    ld = torch.tensor(lens, device=dev)
+    td = torch.tensor(table, device=dev)
+    od = torch.empty_like(qd)
+    max_k = int(lens.max())
+    need = gqa.gqa_attn_decode_varlen_workspace_bytes(w.B, w.Hq, w.Hkv, w.Tq, max_k, w.D, w.window, 0)
+    splits = gqa.gqa_attn_decode_varlen_num_splits(w.B, w.Hq, w.Hkv, w.Tq, max_k, w.D, w.window, 0)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    fn = lambda: gqa.attn_decode_varlen(qd, kd, vd, ld, block_table=td, max_seqlen_k=max_k, window=w.window,
+                                        out=od, workspace=ws)
+    ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after paged decode timing: {gqa.gqa_status_string(st)}")
+    del qd, kd, vd, od, ws
+    torch.cuda.empty_cache()
+    return {"ms_total": ms, "splits": splits, "launches": steps * (1 if splits == 1 else 2)}
+
+
+def varlen_config(w):
+    c = {"workload": w.name, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+         "q_len": f"U[{w.q_lo},{w.q_hi}]", "seed": w.seed, "causal": True, "layout": "token-major packed"}
+    if w.prefix_hi:
+        c["cached_prefix"] = f"U[{w.prefix_lo},{w.prefix_hi}]"
+    return c
+
+
 # ---------------------------------------------------------------- the oracle on the host
 def oracle_sample(w, budget_s: float, threads: int, q=None, k=None, v=None):
     """Time the fp64 oracle on a seeded row sample sized to about budget_s seconds.
@@ -333,7 +400,7 @@ def parse_args(argv=None):
     ap.add_argument("--decode-workload", default="gqa_decode", choices=sorted(gi.WORKLOADS))
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-extensions", action="store_true",
-                    help="skip the sliding-window prefill and decode-chunk measurements")
+                    help="skip the sliding-window, decode-chunk and variable-length measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -520,6 +587,37 @@ def main(argv=None):
                          "frac": achc / peaks["hbm_gbs"], "traffic": None,
                          "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
             "gpu_launches": rc_["launches"]}
+        # variable-length rows: packed prefill, chunked prefill after cached prefixes,
+        # paged decode with per-sequence lengths
+        nsv = max(10, args.steps // 4)
+        for key in ("varlen_prefill", "chunked_prefill"):
+            wv = gi.VARLEN_WORKLOADS[key]
+            rv = measure_varlen(wv, nsv, max(3, args.warmup), world, dev)
+            msv = rv["ms_total"] / nsv
+            achv = varlen_flops(wv) / (msv * 1e-3) / 1e12
+            line[key] = {
+                "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achv,
+                "unit": "TFLOP/s", "ms_per_step": msv,
+                "config": varlen_config(wv) | {"tokens_q": rv["tokens_q"], "tokens_k": rv["tokens_k"]},
+                "roofline": {"bound": "tensor", "achieved": achv, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": achv / peaks["bf16_tflops"], "traffic": None,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                "gpu_launches": rv["launches"]}
+        wp = gi.VARLEN_WORKLOADS["paged_decode"]
+        nsp = max(3, args.steps // 20)
+        rp = measure_paged_decode(wp, nsp, max(3, args.warmup), world, dev)
+        msp = rp["ms_total"] / nsp
+        achp = paged_kv_bytes(wp) / (msp * 1e-3) / 1e9
+        line["paged_decode"] = {
+            "metric": "KV GB/s (every cached key of every sequence)", "value": world * achp, "unit": "GB/s",
+            "ms_per_step": msp,
+            "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "D": wp.D, "Tq": wp.Tq,
+                       "cache_len": f"U[{wp.len_lo},{wp.len_hi}]", "page": wp.page,
+                       "pool": "[pages, page, Hkv, D], seeded random page order", "splits": rp["splits"]},
+            "roofline": {"bound": "hbm", "achieved": achp, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achp / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
+            "gpu_launches": rp["launches"]}
     sampler.stop()
 
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -22,6 +22,7 @@ __all__ = [
     "gqa_attn_decode_ex_workspace_bytes", "gqa_attn_decode_ex_num_splits", "gqa_status_string", "gqa_get_device_error",
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
     "GqaLayout", "gqa_attn_fwd_varlen", "gqa_attn_fwd_varlen_workspace_bytes", "gqa_attn_decode_varlen",
+    "gqa_attn_decode_varlen_workspace_bytes", "gqa_attn_decode_varlen_num_splits",
     "attn_fwd_varlen", "attn_decode_varlen",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
@@ -81,6 +82,10 @@ _lib.gqa_attn_fwd_varlen_workspace_bytes.restype = _sz
 _lib.gqa_attn_fwd_varlen_workspace_bytes.argtypes = [_i32] * 4
 _lib.gqa_attn_fwd_varlen.restype = _i32
 _lib.gqa_attn_fwd_varlen.argtypes = ([_vp] * 9 + [_i32] * 7 + [_lay] * 4 + [_f32, _i32, _vp, _sz, _vp])
+_lib.gqa_attn_decode_varlen_workspace_bytes.restype = _sz
+_lib.gqa_attn_decode_varlen_workspace_bytes.argtypes = [_i32] * 8
+_lib.gqa_attn_decode_varlen_num_splits.restype = _i32
+_lib.gqa_attn_decode_varlen_num_splits.argtypes = [_i32] * 8
 _lib.gqa_attn_decode_varlen.restype = _i32
 _lib.gqa_attn_decode_varlen.argtypes = ([_vp] * 6 + [_i32] * 9 + [_lay] * 2 + [_f32, _i32, _i32, _vp, _sz, _vp])
 _lib.gqa_status_string.restype = ctypes.c_char_p
@@ -178,6 +183,14 @@ def gqa_attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, seqlens_q, 
                                     S, Hq, Hkv, D, rows_q, rows_k, max_seqlen_q, ctypes.byref(lq),
                                     ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
                                     float(softmax_scale), int(window), workspace, workspace_bytes, stream)
+
+
+def gqa_attn_decode_varlen_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window=0, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_varlen_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window, num_splits))
+
+
+def gqa_attn_decode_varlen_num_splits(B, Hq, Hkv, Tq, max_seqlen_k, D, window=0, num_splits=0) -> int:
+    return int(_lib.gqa_attn_decode_varlen_num_splits(B, Hq, Hkv, Tq, max_seqlen_k, D, window, num_splits))
 
 
 def gqa_attn_decode_varlen(q, k_cache, v_cache, o, seqlens_k, block_table, page_size, num_pages,
@@ -423,7 +436,7 @@ def attn_decode_varlen(q, k_cache, v_cache, seqlens_k, *, block_table=None, max_
         max_seqlen_k = max_pages * page_size if max_seqlen_k is None else int(max_seqlen_k)
     if out is None:
         out = torch.empty_like(q)
-    need = gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window, num_splits)
+    need = gqa_attn_decode_varlen_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window, num_splits)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     st = gqa_attn_decode_varlen(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),

@@ -179,15 +179,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const uint32_t fbar = smem_u32(&ctl->full[stage]);
             const uint32_t sK = sbase + stage * L::kStageBytes;
             if (lane == 0) mbar_arrive_expect_tx(fbar, L::kStageBytes);
-            for (int bi = 0; bi < n_box; ++bi) {
-                const int pg = __shfl_sync(0xffffffffu, page, bi);
-                const int rw = __shfl_sync(0xffffffffu, row, bi);
-                if (lane == 0) {
-                    const uint32_t dst = sK + bi * p.box_rows * 128;
-                    for (int c = 0; c < L::kChunks; ++c) {
-                        tma_load_4d(dst + c * L::kChunkBytes, &tm_k, fbar, c * 64, rw, g, pg);
-                        tma_load_4d(dst + L::kTileBytes + c * L::kChunkBytes, &tm_v, fbar, c * 64, rw, g, pg);
-                    }
+            __syncwarp();
+            // lane bi issues the copies of box bi (small pages need many boxes per tile)
+            if (lane < n_box) {
+                const uint32_t dst = sK + lane * p.box_rows * 128;
+                for (int c = 0; c < L::kChunks; ++c) {
+                    tma_load_4d(dst + c * L::kChunkBytes, &tm_k, fbar, c * 64, row, g, page);
+                    tma_load_4d(dst + L::kTileBytes + c * L::kChunkBytes, &tm_v, fbar, c * 64, row, g, page);
                 }
             }
             ++issued[stage];

@@ -100,6 +100,7 @@ int device_sm_count() {
 }
 
 constexpr int kMaxDecodeRows = 16;  // query rows per head the decode path takes (T_q)
+constexpr int kVarlenWaves = 8;     // automatic split target of gqa_attn_decode_varlen
 
 struct SplitPlan {
     int splits, blk_per_split, blk_first, n_blk;
@@ -107,7 +108,10 @@ struct SplitPlan {
 
 // Key blocks [blk_first, n_blk) hold every key some query row can see: with a window
 // the rows of a chunk (positions Tk-Tq .. Tk-1) see nothing before Tk - Tq - window + 1.
-SplitPlan plan_splits(int B, int Hq, int Hkv, int Tq, int Tk, int window, int requested) {
+// `waves`: CTAs per SM the automatic choice aims for. Sequences of different lengths
+// (the varlen call) make CTAs of different lengths; more, shorter CTAs even out the
+// last wave.
+SplitPlan plan_splits(int B, int Hq, int Hkv, int Tq, int Tk, int window, int requested, int waves = 4) {
     SplitPlan sp{};
     sp.n_blk = (Tk + gqa::kTileKeys - 1) / gqa::kTileKeys;
     const int key_lo = window > 0 ? std::max(0, Tk - Tq - window + 1) : 0;
@@ -117,8 +121,8 @@ SplitPlan plan_splits(int B, int Hq, int Hkv, int Tq, int Tk, int window, int re
     const long long units = (long long)B * Hkv * ((G * Tq + 15) / 16);
     int want = requested;
     if (want <= 0) {
-        // about four waves of one CTA per SM, each split at least 8 tiles (1024 keys)
-        const long long target = 4LL * device_sm_count();
+        // about `waves` waves of one CTA per SM, each split at least 8 tiles (1024 keys)
+        const long long target = (long long)waves * device_sm_count();
         want = (int)std::min<long long>((target + units - 1) / units, 1 << 20);
         want = std::min(want, std::max(1, n_range / 8));
     }
@@ -310,6 +314,21 @@ gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void
     return gqa::launch_fwd_varlen(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+int gqa_attn_decode_varlen_num_splits(int B, int Hq, int Hkv, int Tq, int max_seqlen_k, int D, int window,
+                                      int num_splits) {
+    if (check_decode(B, Hq, Hkv, Tq, max_seqlen_k, D, window) != GQA_OK) return 0;
+    return plan_splits(B, Hq, Hkv, Tq, max_seqlen_k, window >= max_seqlen_k ? 0 : window, num_splits,
+                       kVarlenWaves).splits;
+}
+
+size_t gqa_attn_decode_varlen_workspace_bytes(int B, int Hq, int Hkv, int Tq, int max_seqlen_k, int D,
+                                              int window, int num_splits) {
+    if (check_decode(B, Hq, Hkv, Tq, max_seqlen_k, D, window) != GQA_OK) return 0;
+    return ws_bytes_for(plan_splits(B, Hq, Hkv, Tq, max_seqlen_k, window >= max_seqlen_k ? 0 : window,
+                                    num_splits, kVarlenWaves),
+                        (long long)B * Hq * Tq, D);
+}
+
 gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void* v_cache, void* o,
                                   const int* seqlens_k, const int* block_table, int page_size,
                                   int num_pages, int max_pages, int B, int Hq, int Hkv, int Tq,
@@ -340,7 +359,7 @@ gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void
     // The split count is planned for the longest sequence; each sequence shares its
     // own blocks over those splits on the device.
     const SplitPlan sp = plan_splits(B, Hq, Hkv, Tq, max_seqlen_k, window >= max_seqlen_k ? 0 : window,
-                                     num_splits);
+                                     num_splits, kVarlenWaves);
     const long long rows = (long long)B * Hq * Tq;
     if (sp.splits > 1) {
         const size_t need = ws_bytes_for(sp, rows, D);

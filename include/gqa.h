@@ -248,15 +248,21 @@ GQA_API gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void*
  *               are never read; a page number outside [0, num_pages) reads zeros.
  *   max_seqlen_k  >= every L(b); sizes the split plan (and, for a contiguous cache,
  *               the rows the cache must hold).
- *   window, num_splits, workspace   as for gqa_attn_decode_ex; the workspace size is
- *               gqa_attn_decode_ex_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D,
- *               window, num_splits).
+ *   window, num_splits, workspace   as for gqa_attn_decode_ex, but sized by
+ *               gqa_attn_decode_varlen_workspace_bytes with the same arguments: the
+ *               automatic split count (num_splits = 0) aims at twice as many CTAs as
+ *               gqa_attn_decode_ex does, because sequences of different lengths make
+ *               CTAs of different lengths and more, shorter ones even out the last wave.
  * Every L(b) must lie in [Tq, capacity], capacity = max_seqlen_k for a contiguous
  * cache and min(max_seqlen_k, max_pages*page_size) for a paged one. It is checked on
  * the device: a sequence outside that range gets no output and the next
  * gqa_get_device_error() returns GQA_ERR_INVALID_ARGUMENT. Keys past L(b) (the rest
  * of a page, a contiguous cache's unused rows) may hold any bits, NaN included.
  */
+GQA_API size_t gqa_attn_decode_varlen_workspace_bytes(int B, int Hq, int Hkv, int Tq, int max_seqlen_k,
+                                                      int D, int window, int num_splits);
+GQA_API int gqa_attn_decode_varlen_num_splits(int B, int Hq, int Hkv, int Tq, int max_seqlen_k, int D,
+                                              int window, int num_splits);
 GQA_API gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void* v_cache,
                                           void* o, const int* seqlens_k, const int* block_table,
                                           int page_size, int num_pages, int max_pages, int B, int Hq,

@@ -169,3 +169,14 @@ def varlen_dec(gqa, **kw):
 ])
 def test_varlen_decode_rejects_bad_arguments(gqa, kw, status):
     assert varlen_dec(gqa, **kw) == status
+
+
+def test_varlen_decode_split_planning(gqa):
+    # the automatic plan aims at twice the CTAs of the dense plan; explicit requests agree
+    assert gqa.gqa_attn_decode_varlen_num_splits(64, 32, 8, 1, 32768, 128, 0, 0) == 3
+    assert gqa.gqa_attn_decode_ex_num_splits(64, 32, 8, 1, 32768, 128, 0, 0) == 2
+    for s in (1, 4, 7):
+        assert gqa.gqa_attn_decode_varlen_num_splits(4, 8, 2, 1, 4096, 128, 0, s) == \
+            gqa.gqa_attn_decode_ex_num_splits(4, 8, 2, 1, 4096, 128, 0, s)
+    assert gqa.gqa_attn_decode_varlen_workspace_bytes(64, 32, 8, 1, 32768, 128, 0, 1) == 0
+    assert gqa.gqa_attn_decode_varlen_workspace_bytes(64, 32, 8, 17, 32768, 128, 0, 0) == 0  # Tq > 16
