@@ -297,7 +297,7 @@ def paged_kv_bytes(w) -> int:
     return 2 * int(w.lengths().sum()) * w.Hkv * w.D * 2
 
 
-def measure_varlen(w, steps, warmup, world, dev):
+def measure_varlen(w, steps, warmup, world, dev, e2e_steps=0):
     """gqa_attn_fwd_varlen on a packed workload (plan kernel + attention kernel per step)."""
     import torch
     import grouped_query_softmax_b200 as gqa
@@ -316,12 +316,27 @@ def measure_varlen(w, steps, warmup, world, dev):
     st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
     if st != gqa.GQA_OK:
         raise RuntimeError(f"device error after varlen timing: {gqa.gqa_status_string(st)}")
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": 2 * steps, "tokens_q": int(cu_q[-1]),
+           "tokens_k": int(cu_k[-1])}
+    if e2e_steps:
+        hosts = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in (q, k, v)]
+        devs = [x.view(torch.int16) for x in (qd, kd, vd)]
+        oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+
+        def e2e_step():
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            fn()
+            oh.copy_(od.view(torch.int16), non_blocking=True)
+        e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
+        res.update(e2e_ms_total=e2e_ms, e2e_steps=e2e_steps, h2d_bytes=int(q.nbytes + k.nbytes + v.nbytes),
+                   d2h_bytes=int(q.nbytes))
     del qd, kd, vd, od, ws
     torch.cuda.empty_cache()
-    return {"ms_total": ms, "launches": 2 * steps, "tokens_q": int(cu_q[-1]), "tokens_k": int(cu_k[-1])}
+    return res
 
 
-def measure_paged_decode(w, steps, warmup, world, dev):
+def measure_paged_decode(w, steps, warmup, world, dev, e2e_steps=0):
     """gqa_attn_decode_varlen over the paged pool of a PagedDecodeWorkload."""
     import torch
     import grouped_query_softmax_b200 as gqa
@@ -340,9 +355,24 @@ def measure_paged_decode(w, steps, warmup, world, dev):
     st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
     if st != gqa.GQA_OK:
         raise RuntimeError(f"device error after paged decode timing: {gqa.gqa_status_string(st)}")
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "splits": splits,
+           "launches": steps * (1 if splits == 1 else 2)}
+    if e2e_steps:
+        hosts = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in (q, kp, vp)]
+        devs = [x.view(torch.int16) for x in (qd, kd, vd)]
+        oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+
+        def e2e_step():
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            fn()
+            oh.copy_(od.view(torch.int16), non_blocking=True)
+        e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
+        res.update(e2e_ms_total=e2e_ms, e2e_steps=e2e_steps, h2d_bytes=int(q.nbytes + kp.nbytes + vp.nbytes),
+                   d2h_bytes=int(q.nbytes))
     del qd, kd, vd, od, ws
     torch.cuda.empty_cache()
-    return {"ms_total": ms, "splits": splits, "launches": steps * (1 if splits == 1 else 2)}
+    return res
 
 
 def varlen_config(w):
@@ -396,7 +426,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gqa_prefill", choices=sorted(gi.WORKLOADS))
+    ap.add_argument("--workload", default="gqa_prefill", choices=sorted(gi.WORKLOADS) + sorted(gi.VARLEN_WORKLOADS),
+                    help="main workload (a varlen or paged one is measured alone, e.g. for profiling)")
     ap.add_argument("--decode-workload", default="gqa_decode", choices=sorted(gi.WORKLOADS))
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-extensions", action="store_true",
@@ -405,7 +436,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--batch", type=int, default=0,
-                    help="override the main workload's batch size (for profiling a smaller case)")
+                    help="override the main workload's batch size / sequence count (for profiling a smaller case)")
     return ap.parse_args(argv)
 
 
@@ -435,6 +466,8 @@ def reference_arm(args, rank, world):
     """The oracle as the reference arm: rank 0 alone runs it; other ranks exit 0."""
     if rank != 0:
         return
+    if args.workload not in gi.WORKLOADS:
+        raise SystemExit("--impl reference times the oracle on the dense workloads only")
     w = gi.WORKLOADS[args.workload]
     threads = cpu_threads()
     q, k, v = w.make()
@@ -465,6 +498,56 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def varlen_main(args, rank, world, local, dev, peaks, peak_src):
+    """A variable-length or paged workload as the main line (profiling and focused runs)."""
+    import dataclasses
+    w = gi.VARLEN_WORKLOADS[args.workload]
+    if args.batch > 0:
+        field = "B" if isinstance(w, gi.PagedDecodeWorkload) else "S"
+        w = dataclasses.replace(w, **{field: args.batch}, name=f"{w.name} ({field} {args.batch})")
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local])
+    sampler.start()
+    time.sleep(0.2)
+    if isinstance(w, gi.PagedDecodeWorkload):
+        r = measure_paged_decode(w, args.steps, args.warmup, world, dev, args.e2e_steps)
+        work, unit, scale = paged_kv_bytes(w), "GB/s", 1e9
+        metric = "GQA paged decode KV GB/s on 1 B200, % of roofline"
+        config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Tq": w.Tq,
+                  "cache_len": f"U[{w.len_lo},{w.len_hi}]", "page": w.page, "splits": r["splits"]}
+        peak, bound, src = peaks["hbm_gbs"], "hbm", f"{peak_src} hbm_gbs (copy, read+write bytes)"
+        kernel = "gqa_decode_sm100_kernel<varlen> + gqa_decode_combine_kernel"
+    else:
+        r = measure_varlen(w, args.steps, args.warmup, world, dev, args.e2e_steps)
+        work, unit, scale = varlen_flops(w), "TFLOP/s", 1e12
+        metric = "GQA varlen prefill TFLOP/s on 1 B200, % of roofline"
+        config = varlen_config(w) | {"tokens_q": r["tokens_q"], "tokens_k": r["tokens_k"]}
+        peak, bound, src = peaks["bf16_tflops"], "tensor", f"{peak_src} bf16_tflops (burst)"
+        kernel = "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen>"
+    ms_step = r["ms_total"] / args.steps
+    achieved = work / (ms_step * 1e-3) / scale
+    clocks = sampler.summary(r["t0"], r["t1"])
+    sampler.stop()
+    line = {"metric": metric, "value": world * achieved, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config | {"l2": "inputs larger than L2 (no flush)",
+                                "parallelism": f"dp{world} (independent problems per rank)"},
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": None, "peak_source": src, "kernel": kernel},
+            "gpu_launches": r["launches"], "clocks": clocks}
+    if args.e2e_steps:
+        e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
+        line["e2e"] = {"value": world * work / (e2e_ms * 1e-3) / scale, "unit": unit,
+                       "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"],
+                       "ms_per_step": e2e_ms, "steps": r["e2e_steps"]}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
@@ -484,6 +567,8 @@ def main(argv=None):
     import grouped_query_softmax_b200 as gqa  # noqa: F401  (fails loudly without libgqa.so)
 
     peaks, peak_src = load_peaks()
+    if args.workload in gi.VARLEN_WORKLOADS:
+        return varlen_main(args, rank, world, local, dev, peaks, peak_src)
     w = gi.WORKLOADS[args.workload]
     if args.batch > 0:
         import dataclasses
@@ -600,7 +685,8 @@ def main(argv=None):
                 "unit": "TFLOP/s", "ms_per_step": msv,
                 "config": varlen_config(wv) | {"tokens_q": rv["tokens_q"], "tokens_k": rv["tokens_k"]},
                 "roofline": {"bound": "tensor", "achieved": achv, "peak": peaks["bf16_tflops"],
-                             "unit": "TFLOP/s", "frac": achv / peaks["bf16_tflops"], "traffic": None,
+                             "unit": "TFLOP/s", "frac": achv / peaks["bf16_tflops"],
+                             "traffic": load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
                 "gpu_launches": rv["launches"]}
         wp = gi.VARLEN_WORKLOADS["paged_decode"]
@@ -615,7 +701,8 @@ def main(argv=None):
                        "cache_len": f"U[{wp.len_lo},{wp.len_hi}]", "page": wp.page,
                        "pool": "[pages, page, Hkv, D], seeded random page order", "splits": rp["splits"]},
             "roofline": {"bound": "hbm", "achieved": achp, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achp / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achp / peaks["hbm_gbs"],
+                         "traffic": load_traffic("gqa_decode_sm100_kernel_varlen", wp.name),
                          "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
             "gpu_launches": rp["launches"]}
     sampler.stop()
