@@ -26,6 +26,7 @@ _LIB = os.path.join(_HERE, "libgqa_inputs.so")
 TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
 # streams of the integer draws: query-chunk lengths, cached-prefix lengths, page order
 STREAM_LEN, STREAM_PREFIX, STREAM_PAGES = 3, 4, 5
+TENSOR_DO = 6  # the output gradient dO of the backward pass, N(0,1) bf16 like Q/K/V
 
 
 def build(force: bool = False) -> str:
@@ -139,6 +140,10 @@ class Workload:
     @property
     def kv_shape(self):
         return (self.B, self.Hkv, self.Tk, self.D)
+
+    def make_dout(self, threads: int | None = None):
+        """The output gradient dO for this workload's backward pass ([B, Hq, Tq, D] bf16 bits)."""
+        return normal_bf16(self.seed, TENSOR_DO, self.q_shape, threads=threads)
 
     def make(self, threads: int | None = None, q_out=None, k_out=None, v_out=None):
         """Generate (q, k, v) bf16 bit arrays for this workload."""

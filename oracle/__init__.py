@@ -45,6 +45,10 @@ def _bind(lib):
     lib.gqa_oracle_rows_window.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                            ll, ll, ll, ll, ll, ll, ctypes.c_double, i32,
                                            vp, ll, vp, vp, i32]
+    lib.gqa_oracle_bwd.restype = i32
+    lib.gqa_oracle_bwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                   ll, ll, ll, ll, ll, ll, ctypes.c_double, i32,
+                                   vp, vp, vp, i32]
     return lib
 
 
@@ -122,3 +126,36 @@ def load_variant(path: str):
     Used only by the pin tests, which compile copies of the oracle with a
     planted mistake and check that some pin catches each one."""
     return _bind(ctypes.CDLL(path))
+
+
+def attention_bwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarray, Tk: int | None = None,
+                  scale: float | None = None, window: int = 0, threads: int | None = None, lib=None):
+    """fp64 gradients (dq, dk, dv) of causal GQA attention for the output gradient ``dout``.
+
+    q and dout: uint16 [B, H_q, T_q, D] (the same layout); k, v: uint16 [B, H_kv, T_cap, D]
+    with the first ``Tk`` rows used. Returns float64 dq [B, H_q, T_q, D] and dk, dv
+    [B, H_kv, Tk, D]; a KV head's dk and dv sum over all the query heads that read it.
+    """
+    B, Hq, Tq, D = q.shape
+    Hkv, Tcap = k.shape[1], k.shape[2]
+    if dout.shape != q.shape or v.shape != k.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("shape mismatch between q, k, v and dout")
+    Tk = Tcap if Tk is None else int(Tk)
+    q_sb, q_sh = _plane_strides(q, "q")
+    d_sb, d_sh = _plane_strides(dout, "dout")
+    if (d_sb, d_sh) != (q_sb, q_sh):
+        raise ValueError("dout must have q's strides")
+    k_sb, k_sh = _plane_strides(k, "k")
+    v_sb, v_sh = _plane_strides(v, "v")
+    dq = np.empty((B, Hq, Tq, D), dtype=np.float64)
+    dk = np.empty((B, Hkv, Tk, D), dtype=np.float64)
+    dv = np.empty((B, Hkv, Tk, D), dtype=np.float64)
+    rc = (lib or _load()).gqa_oracle_bwd(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, Hq, Hkv, Tq, Tk, D,
+        q_sb, q_sh, k_sb, k_sh, v_sb, v_sh, float(scale) if scale else 0.0, int(window),
+        dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(threads or default_threads()))
+    if rc == 1:
+        raise ValueError("oracle rejected the arguments (H_q % H_kv != 0, T_q > T_k ...)")
+    if rc != 0:
+        raise MemoryError("oracle allocation failed")
+    return dq, dk, dv

@@ -186,3 +186,146 @@ int gqa_oracle_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
     return gqa_oracle_rows_window(q, k, v, B, Hq, Hkv, Tq, Tk, D, q_sb, q_sh, k_sb, k_sh, v_sb, v_sh,
                                   scale, 0, rows, n_rows, out, lse, n_threads);
 }
+
+/*
+ * Gradients of the same attention, for the training side (fp64, test infrastructure).
+ *
+ * The pages only say that FlashAttention's backward recomputes the scores, which adds
+ * FLOPs ("长上下文与高效注意力：研究账本", section FlashAttention). What it computes is
+ * the derivative of the o_a definition above. With P_ij the softmax weights of row i over its
+ * visible keys j, s_ij = scale <q_i, k_j>, and dO = dL/dO for a scalar loss L:
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   dS_ij = P_ij (dP_ij - sum_l P_il dP_il)         (softmax Jacobian applied to dP)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i
+ * A KV head's dK and dV sum over every query head a with g(a) = g, and over every row.
+ * One (b, g) plane per work item, rows in order, so the fp64 sums are deterministic.
+ */
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    int B, Hq, Hkv, Tq, Tk, D;
+    long long q_sb, q_sh, k_sb, k_sh, v_sb, v_sh; /* dout uses q's strides */
+    double scale;
+    int window;
+    double *dq, *dk, *dv; /* [B,Hq,Tq,D], [B,Hkv,Tk,D], [B,Hkv,Tk,D], contiguous */
+    long long next;
+} oracle_bwd_job;
+
+static void oracle_bwd_plane(const oracle_bwd_job* J, long long bg, double* p, double* dp, double* qd,
+                             double* dod) {
+    const int D = J->D;
+    const long long Tk = J->Tk, Tq = J->Tq;
+    const long long b = bg / J->Hkv, g = bg % J->Hkv;
+    const long long group = J->Hq / J->Hkv;
+    const uint16_t* kplane = J->k + b * J->k_sb + g * J->k_sh;
+    const uint16_t* vplane = J->v + b * J->v_sb + g * J->v_sh;
+    double* dk = J->dk + bg * Tk * D;
+    double* dv = J->dv + bg * Tk * D;
+    for (long long e = 0; e < Tk * D; ++e) dk[e] = dv[e] = 0.0;
+    for (long long a = g * group; a < (g + 1) * group; ++a) {
+        for (long long i = 0; i < Tq; ++i) {
+            const long long pos = (Tk - Tq) + i;
+            const long long first = (J->window > 0 && pos - J->window + 1 > 0) ? pos - J->window + 1 : 0;
+            const uint16_t* qrow = J->q + b * J->q_sb + a * J->q_sh + i * D;
+            const uint16_t* dorow = J->dout + b * J->q_sb + a * J->q_sh + i * D;
+            for (int d = 0; d < D; ++d) {
+                qd[d] = bf16_to_double(qrow[d]);
+                dod[d] = bf16_to_double(dorow[d]);
+            }
+            /* P: softmax of the scaled scores over the visible keys */
+            double m = -INFINITY;
+            for (long long j = first; j <= pos; ++j) {
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += qd[d] * bf16_to_double(kplane[j * D + d]);
+                p[j] = J->scale * acc;
+                if (p[j] > m) m = p[j];
+            }
+            double l = 0.0;
+            for (long long j = first; j <= pos; ++j) {
+                p[j] = exp(p[j] - m);
+                l += p[j];
+            }
+            for (long long j = first; j <= pos; ++j) p[j] /= l;
+            /* dP and the row term sum_l P_il dP_il */
+            double rowterm = 0.0;
+            for (long long j = first; j <= pos; ++j) {
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += dod[d] * bf16_to_double(vplane[j * D + d]);
+                dp[j] = acc;
+                rowterm += p[j] * dp[j];
+            }
+            double* dqrow = J->dq + ((b * J->Hq + a) * Tq + i) * D;
+            for (int d = 0; d < D; ++d) dqrow[d] = 0.0;
+            for (long long j = first; j <= pos; ++j) {
+                const double ds = p[j] * (dp[j] - rowterm);
+                for (int d = 0; d < D; ++d) {
+                    dqrow[d] += J->scale * ds * bf16_to_double(kplane[j * D + d]);
+                    dk[j * D + d] += J->scale * ds * qd[d];
+                    dv[j * D + d] += p[j] * dod[d];
+                }
+            }
+        }
+    }
+}
+
+static void* oracle_bwd_worker(void* arg) {
+    oracle_bwd_job* J = (oracle_bwd_job*)arg;
+    double* p = (double*)malloc(sizeof(double) * (size_t)J->Tk);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)J->Tk);
+    double* qd = (double*)malloc(sizeof(double) * (size_t)J->D);
+    double* dod = (double*)malloc(sizeof(double) * (size_t)J->D);
+    void* ret = NULL;
+    if (!p || !dp || !qd || !dod) {
+        ret = (void*)1;
+    } else {
+        for (;;) {
+            const long long bg = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+            if (bg >= (long long)J->B * J->Hkv) break;
+            oracle_bwd_plane(J, bg, p, dp, qd, dod);
+        }
+    }
+    free(p);
+    free(dp);
+    free(qd);
+    free(dod);
+    return ret;
+}
+
+/*
+ * dq [B,Hq,Tq,D], dk and dv [B,Hkv,Tk,D] (doubles, contiguous) of the attention of q over the
+ * first Tk keys of k/v, for the output gradient dout (bf16 bits, q's layout).
+ * scale <= 0 selects 1/sqrt(D); window as for gqa_oracle_rows_window.
+ * Returns 0 on success, 1 on invalid arguments, 2 on allocation failure.
+ */
+int gqa_oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int B,
+                   int Hq, int Hkv, int Tq, int Tk, int D, long long q_sb, long long q_sh, long long k_sb,
+                   long long k_sh, long long v_sb, long long v_sh, double scale, int window, double* dq,
+                   double* dk, double* dv, int n_threads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return 1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || D <= 0) return 1;
+    if (Hq % Hkv != 0 || Tq > Tk) return 1;
+    oracle_bwd_job J;
+    J.q = q; J.k = k; J.v = v; J.dout = dout;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Tq = Tq; J.Tk = Tk; J.D = D;
+    J.q_sb = q_sb; J.q_sh = q_sh; J.k_sb = k_sb; J.k_sh = k_sh; J.v_sb = v_sb; J.v_sh = v_sh;
+    J.scale = scale > 0.0 ? scale : 1.0 / sqrt((double)D);
+    J.window = window;
+    J.dq = dq; J.dk = dk; J.dv = dv; J.next = 0;
+    if (n_threads <= 1) return oracle_bwd_worker(&J) ? 2 : 0;
+    if (n_threads > 512) n_threads = 512;
+    pthread_t th[512];
+    int started[512], any = 0, rc = 0;
+    for (int t = 0; t < n_threads; ++t) {
+        started[t] = pthread_create(&th[t], NULL, oracle_bwd_worker, &J) == 0;
+        any |= started[t];
+    }
+    for (int t = 0; t < n_threads; ++t) {
+        if (!started[t]) continue;
+        void* ret = NULL;
+        pthread_join(th[t], &ret);
+        if (ret) rc = 2;
+    }
+    if (!any) rc = oracle_bwd_worker(&J) ? 2 : 0;
+    return rc;
+}
