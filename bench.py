@@ -35,7 +35,7 @@ import numpy as np  # noqa: E402
 import gqa_inputs as gi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["grouped_query_softmax_b200/csrc/fwd_sm100.cuh",
+KERNEL_SOURCES = ["grouped_query_softmax_b200/csrc/fwd_sm100.cuh", "grouped_query_softmax_b200/csrc/bwd_sm100.cuh",
                   "grouped_query_softmax_b200/csrc/decode_sm100.cuh",
                   "grouped_query_softmax_b200/csrc/sm100_ptx.cuh"]
 

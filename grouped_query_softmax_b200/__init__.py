@@ -23,6 +23,7 @@ __all__ = [
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
     "GqaLayout", "gqa_attn_fwd_varlen", "gqa_attn_fwd_varlen_workspace_bytes", "gqa_attn_decode_varlen",
     "gqa_attn_decode_varlen_workspace_bytes", "gqa_attn_decode_varlen_num_splits",
+    "gqa_attn_bwd", "gqa_attn_bwd_workspace_bytes", "attn_bwd",
     "attn_fwd_varlen", "attn_decode_varlen",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
@@ -88,6 +89,10 @@ _lib.gqa_attn_decode_varlen_num_splits.restype = _i32
 _lib.gqa_attn_decode_varlen_num_splits.argtypes = [_i32] * 8
 _lib.gqa_attn_decode_varlen.restype = _i32
 _lib.gqa_attn_decode_varlen.argtypes = ([_vp] * 6 + [_i32] * 9 + [_lay] * 2 + [_f32, _i32, _i32, _vp, _sz, _vp])
+_lib.gqa_attn_bwd_workspace_bytes.restype = _sz
+_lib.gqa_attn_bwd_workspace_bytes.argtypes = [_i32] * 6
+_lib.gqa_attn_bwd.restype = _i32
+_lib.gqa_attn_bwd.argtypes = [_vp] * 9 + [_i32] * 6 + [_ll] * 4 + [_f32, _vp, _sz, _vp]
 _lib.gqa_status_string.restype = ctypes.c_char_p
 _lib.gqa_status_string.argtypes = [_i32]
 _lib.gqa_get_device_error.restype = _i32
@@ -203,6 +208,17 @@ def gqa_attn_decode_varlen(q, k_cache, v_cache, o, seqlens_k, block_table, page_
                                        num_pages, max_pages, B, Hq, Hkv, Tq, max_seqlen_k, D,
                                        ctypes.byref(lk), ctypes.byref(lv), float(softmax_scale),
                                        int(window), int(num_splits), workspace, workspace_bytes, stream)
+
+
+def gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Tq, Tk, D) -> int:
+    return int(_lib.gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Tq, Tk, D))
+
+
+def gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                 softmax_scale=0.0, workspace=None, workspace_bytes=0, stream=None) -> int:
+    """C ``gqa_attn_bwd``: dq, dk, dv of the causal GQA forward for the output gradient dout."""
+    return _lib.gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                             float(softmax_scale), workspace, workspace_bytes, stream)
 
 
 def gqa_status_string(status: int) -> str:
@@ -447,3 +463,38 @@ def attn_decode_varlen(q, k_cache, v_cache, seqlens_k, *, block_table=None, max_
     if st != GQA_OK:
         raise GqaError(st, "gqa_attn_decode_varlen")
     return out
+
+
+def attn_bwd(q, k, v, o, dout, lse, *, Tk=None, scale=None, dq=None, dk=None, dv=None, workspace=None,
+             stream=None):
+    """Gradients (dq, dk, dv) of ``attn_fwd(q, k, v)`` for the output gradient ``dout``.
+
+    o and lse are the forward's output and its log-sum-exp (``attn_fwd(..., return_lse=True)``);
+    q, o, dout [B,Hq,Tq,D] contiguous; k, v [B,Hkv,T_cap,D] (first Tk rows). dk and dv are
+    [B,Hkv,Tk,D]; a KV head's gradient sums over the query heads that read it.
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check_bf16_cuda(t, n)
+    for t, n in ((q, "q"), (o, "o"), (dout, "dout")):
+        if not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{n} must be contiguous and shaped like q")
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise TypeError("lse must be a contiguous fp32 CUDA tensor")
+    B, Hq, Tq, D = q.shape
+    Hkv = k.shape[1]
+    Tk = k.shape[2] if Tk is None else int(Tk)
+    k_sb, k_sh = _plane_strides(k, "k")
+    v_sb, v_sh = _plane_strides(v, "v")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty((B, Hkv, Tk, D), dtype=q.dtype, device=q.device) if dk is None else dk
+    dv = torch.empty((B, Hkv, Tk, D), dtype=q.dtype, device=q.device) if dv is None else dv
+    need = gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Tq, Tk, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = gqa_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                      float(scale or 0.0), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_bwd")
+    return dq, dk, dv

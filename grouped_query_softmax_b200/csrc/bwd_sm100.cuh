@@ -1,0 +1,479 @@
+// Causal grouped-query attention backward for sm_100a: dQ, dK, dV.
+//
+// The gradients of o_a = softmax(Q_a K_g^T * scale + M) V_g ("注意力家族", section
+// 统一记号) for an output gradient dO, with P_ij the softmax weights of row i:
+//   dV_j = sum_i P_ij dO_i,  dP_ij = <dO_i, v_j>,  dS_ij = P_ij (dP_ij - D_i),
+//   D_i = sum_j P_ij dP_ij = <dO_i, O_i>,  dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,
+// with a KV head's dK and dV summed over the G query heads that read it. As in the
+// FlashAttention backward ("长上下文与高效注意力：研究账本", section FlashAttention: the backward
+// recomputes, adding FLOPs) P is recomputed from Q, K and the forward's log-sum-exp; the
+// T_q x T_k matrices never reach HBM.
+//
+// B200 mapping. A CTA owns one 128-key block j of one KV head g of one batch b and walks
+// every (query head a of the group, 128-row query tile i) that sees those keys, so dK and
+// dV accumulate in TMEM for the whole group without atomics. Per step, with K_j and V_j
+// resident in shared memory:
+//   S^T  = K_j Q_i^T      (tcgen05, TMEM; lanes = keys)
+//   P^T  = 2^(S^T scale log2e - LSE_i log2e), causal mask on the diagonal tiles (bf16, in place)
+//   dP^T = V_j dO_i^T     (TMEM)
+//   dV  += P^T dO_i       (A from TMEM)
+//   dS^T = P^T (dP^T - D_i)  -> shared memory, bf16, [keys][rows]
+//   dK  += dS^T Q_i       (A = dS^T, K-major)
+//   dQ_i = dS K_j         (A = the same buffer read M-major), added into an fp32 dQ buffer
+// Warps: 0 TMA producer (K_j, V_j once; Q_i and dO_i through a 2-slot ring), 1 tcgen05
+// issuer, 2 TMEM allocation, 4-7 the P / dS warpgroup (thread t owns key row t and keeps
+// its 128 probabilities in registers), 8-11 the dQ warpgroup (thread t owns query row t of
+// the dQ tile; adds it to the fp32 buffer with vector reductions) and, at the end, the dK
+// and dV epilogue. TMEM (512 columns at D = 128): S^T | dP^T, later dQ | dV | dK.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+
+constexpr int kBwdKeys = 128;     // keys per CTA
+constexpr int kBwdRows = 128;     // query rows per step
+constexpr int kBwdThreads = 384;
+// Register split (setmaxnreg): 384 x 168 at launch = 128 x (136 + 240 + 128).
+constexpr int kBwdLaunchRegs = 168;
+constexpr int kBwdCtlRegs = 136;
+constexpr int kBwdPRegs = 240;
+constexpr int kBwdDqRegs = 128;
+static_assert(128 * (kBwdCtlRegs + kBwdPRegs + kBwdDqRegs) <= kBwdThreads * kBwdLaunchRegs,
+              "register split exceeds the launch allocation");
+
+struct BwdParams {
+    int B, Hq, Hkv, Tq, Tk, G;
+    int n_qt;       // ceil(Tq / 128)
+    int tq_pad;     // n_qt * 128: row stride of lse2 and dvec
+    float scale;
+    float scale_log2;     // scale * log2(e)
+    const float* lse2;    // [B, Hq, tq_pad]: the forward's LSE * log2(e); +inf past Tq
+    const float* dvec;    // [B, Hq, tq_pad]: <dO_i, O_i>; 0 past Tq
+    float* dq_acc;        // [B, Hq, Tq, D] fp32, zeroed by the prep kernel
+    __nv_bfloat16* dk;    // [B, Hkv, Tk, D]
+    __nv_bfloat16* dv;    // [B, Hkv, Tk, D]
+    uint32_t* err;
+    unsigned long long timeout_ns;
+};
+
+template <int D>
+struct BwdSmem {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kChunks * kChunkBytes;  // one [128][D] bf16 tile
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kTileBytes;
+    static constexpr int kRingOff = 2 * kTileBytes;        // 2 slots of (Q_i, dO_i)
+    static constexpr int kSlotBytes = 2 * kTileBytes;
+    static constexpr int kDsOff = kRingOff + 2 * kSlotBytes;  // dS^T [128 keys][128 rows] bf16
+    static constexpr int kDsBytes = 2 * kChunkBytes;
+    static constexpr int kCtlOff = kDsOff + kDsBytes;
+    struct Ctl {
+        uint64_t kv_full;
+        uint64_t qdo_full[2];
+        uint64_t qdo_empty[2];
+        uint64_t s_full, p_full, dp_full, ds_full, ds_empty, dq_full, dq_empty, dkdv_full;
+        uint64_t drain;
+        uint32_t tmem_base;
+        uint32_t abort;
+    };
+    static constexpr int kBytes = kCtlOff + (int)sizeof(Ctl) + 1024;
+};
+
+// First 128-row query tile with a row that sees key block j (row r sees key k iff
+// k <= Tk - Tq + r).
+__device__ __forceinline__ int bwd_first_tile(int j, int Tq, int Tk) {
+    const int r = j * kBwdKeys - (Tk - Tq);
+    return r > 0 ? r / kBwdRows : 0;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float4 ldg_f4(const float* p) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    gqa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const BwdParams p) {
+    using L = BwdSmem<D>;
+    using Ctl = typename L::Ctl;
+    constexpr int kTileBytes = L::kTileBytes;
+    constexpr int kChunkBytes = L::kChunkBytes;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t sbase = raw_addr + pad;
+    const uint32_t sK = sbase + L::kKOff;
+    const uint32_t sV = sbase + L::kVOff;
+    const uint32_t sRing = sbase + L::kRingOff;
+    const uint32_t sDS = sbase + L::kDsOff;
+    Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtlOff);
+    volatile uint32_t* abort_flag = &ctl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bg = blockIdx.x;  // b * Hkv + g
+    const int b = bg / p.Hkv;
+    const int g = bg - b * p.Hkv;
+    const int j = blockIdx.y;   // key block; low j first (they have the most work)
+    const int off = p.Tk - p.Tq;
+    const int i0 = bwd_first_tile(j, p.Tq, p.Tk);
+    const int items = p.G * (p.n_qt - i0);  // (query tile, head) steps, tile-major
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&ctl->kv_full), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&ctl->qdo_full[s]), 1);
+            mbar_init(smem_u32(&ctl->qdo_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&ctl->s_full), 1);
+        mbar_init(smem_u32(&ctl->p_full), 128);
+        mbar_init(smem_u32(&ctl->dp_full), 1);
+        mbar_init(smem_u32(&ctl->ds_full), 128);
+        mbar_init(smem_u32(&ctl->ds_empty), 1);
+        mbar_init(smem_u32(&ctl->dq_full), 1);
+        mbar_init(smem_u32(&ctl->dq_empty), 128);
+        mbar_init(smem_u32(&ctl->dkdv_full), 1);
+        mbar_init(smem_u32(&ctl->drain), 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 32) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_do);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t tS = tmem;                    // S^T, P^T (bf16 in the first 64 columns)
+    const uint32_t tDP = tmem + 128u;            // dP^T, then dQ
+    const uint32_t tDV = tmem + 256u;            // dV (D columns)
+    const uint32_t tDK = tmem + 256u + (uint32_t)D;  // dK (D columns)
+
+    if (warp < 4) setmaxnreg_dec<kBwdCtlRegs>();
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            const uint32_t kvbar = smem_u32(&ctl->kv_full);
+            mbar_arrive_expect_tx(kvbar, 2 * kTileBytes);
+            for (int c = 0; c < L::kChunks; ++c) {
+                tma_load_4d(sK + c * kChunkBytes, &tm_k, kvbar, c * 64, j * kBwdKeys, g, b);
+                tma_load_4d(sV + c * kChunkBytes, &tm_v, kvbar, c * 64, j * kBwdKeys, g, b);
+            }
+            uint32_t issued[2] = {0u, 0u};
+            for (int w = 0; w < items && ok; ++w) {
+                const int slot = w & 1;
+                const int i = i0 + w / p.G;
+                const int a = g * p.G + (w - (w / p.G) * p.G);
+                if (w >= 2 && !(ok = mbar_wait_bounded(smem_u32(&ctl->qdo_empty[slot]), ((w >> 1) - 1) & 1u,
+                                                       abort_flag, p.err, p.timeout_ns)))
+                    break;
+                const uint32_t fbar = smem_u32(&ctl->qdo_full[slot]);
+                const uint32_t sQ = sRing + slot * L::kSlotBytes;
+                mbar_arrive_expect_tx(fbar, 2 * kTileBytes);
+                for (int c = 0; c < L::kChunks; ++c) {
+                    tma_load_4d(sQ + c * kChunkBytes, &tm_q, fbar, c * 64, i * kBwdRows, a, b);
+                    tma_load_4d(sQ + kTileBytes + c * kChunkBytes, &tm_do, fbar, c * 64, i * kBwdRows, a, b);
+                }
+                ++issued[slot];
+            }
+            if (*abort_flag) {
+                mbar_wait_drain(kvbar, 0, p.timeout_ns);
+                for (int s = 0; s < 2; ++s)
+                    if (issued[s]) mbar_wait_drain(smem_u32(&ctl->qdo_full[s]), (issued[s] - 1u) & 1u, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ tcgen05 issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_t = umma_idesc_bf16(kBwdKeys, kBwdRows, 0, 0);  // S^T, dP^T
+            constexpr uint32_t idesc_kv = umma_idesc_bf16(kBwdKeys, D, 0, 1);       // dV, dK
+            constexpr uint32_t idesc_q = umma_idesc_bf16(kBwdRows, D, 1, 1);        // dQ
+            const uint64_t dK_kmaj = umma_desc_sw128(sK, 16, 1024);
+            const uint64_t dV_kmaj = umma_desc_sw128(sV, 16, 1024);
+            const uint64_t dK_nmaj = umma_desc_sw128(sK, kChunkBytes, 1024);
+            const uint64_t dS_kmaj = umma_desc_sw128(sDS, 16, 1024);
+            const uint64_t dS_mmaj = umma_desc_sw128(sDS, kChunkBytes, 1024);
+            bool ok = mbar_wait_bounded(smem_u32(&ctl->kv_full), 0, abort_flag, p.err, p.timeout_ns);
+            tc_fence_after_sync();
+            for (int w = 0; w < items && ok; ++w) {
+                const int slot = w & 1;
+                const uint32_t ph = w & 1;
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->qdo_full[slot]), (w >> 1) & 1u, abort_flag, p.err,
+                                             p.timeout_ns)))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t sQ = sRing + slot * L::kSlotBytes;
+                const uint32_t sDO = sQ + kTileBytes;
+                const uint64_t dQ_kmaj = umma_desc_sw128(sQ, 16, 1024);
+                const uint64_t dDO_kmaj = umma_desc_sw128(sDO, 16, 1024);
+                const uint64_t dQ_nmaj = umma_desc_sw128(sQ, kChunkBytes, 1024);
+                const uint64_t dDO_nmaj = umma_desc_sw128(sDO, kChunkBytes, 1024);
+                // S^T = K_j Q_i^T: M = 128 keys, N = 128 rows, K = D in steps of 16
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tS, dK_kmaj + ko, dQ_kmaj + ko, idesc_t, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(smem_u32(&ctl->s_full));
+                // dP^T = V_j dO_i^T into the dQ columns, once the previous dQ has been read
+                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->dq_empty), (w - 1) & 1u, abort_flag, p.err,
+                                                      p.timeout_ns)))
+                    break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tDP, dV_kmaj + ko, dDO_kmaj + ko, idesc_t, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(smem_u32(&ctl->dp_full));
+                // dV += P^T dO_i: A = P^T (bf16 pairs in TMEM), K = 128 query rows
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->p_full), ph, abort_flag, p.err, p.timeout_ns))) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kBwdRows / 16; ++kk)
+                    tc_mma_ts(tDV, tS + kk * 8, dDO_nmaj + (uint64_t)((kk * 2048) >> 4), idesc_kv,
+                              (w > 0 || kk > 0) ? 1u : 0u);
+                // dK += dS^T Q_i and dQ_i = dS K_j, once dS^T is in shared memory
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), ph, abort_flag, p.err, p.timeout_ns))) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kBwdRows / 16; ++kk) {
+                    const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+                    tc_mma_ss(tDK, dS_kmaj + ko, dQ_nmaj + (uint64_t)((kk * 2048) >> 4), idesc_kv,
+                              (w > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kBwdKeys / 16; ++kk)
+                    tc_mma_ss(tDP, dS_mmaj + (uint64_t)((kk * 2048) >> 4), dK_nmaj + (uint64_t)((kk * 2048) >> 4),
+                              idesc_q, kk > 0 ? 1u : 0u);
+                tc_commit(smem_u32(&ctl->dq_full));
+                tc_commit(smem_u32(&ctl->ds_empty));
+                tc_commit(smem_u32(&ctl->qdo_empty[slot]));
+            }
+            if (ok) tc_commit(smem_u32(&ctl->dkdv_full));
+            if (*abort_flag) {
+                tc_commit(smem_u32(&ctl->drain));
+                mbar_wait_drain(smem_u32(&ctl->drain), 0, p.timeout_ns);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ P and dS
+        setmaxnreg_inc<kBwdPRegs>();
+        const int t = (warp - 4) * 32 + lane;              // key row = TMEM lane
+        const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
+        const int kabs = j * kBwdKeys + t;                 // this thread's key position
+        bool ok = true;
+        for (int w = 0; w < items && ok; ++w) {
+            const uint32_t ph = w & 1;
+            const int i = i0 + w / p.G;
+            const int a = g * p.G + (w - (w / p.G) * p.G);
+            const size_t vrow = ((size_t)b * p.Hq + a) * p.tq_pad + (size_t)i * kBwdRows;
+            const float* lse2 = p.lse2 + vrow;
+            const float* dvec = p.dvec + vrow;
+            // column c (query row i*128 + c) sees this key iff c >= lim
+            const int lim = kabs - (off + i * kBwdRows);
+            const bool diag = j * kBwdKeys + kBwdKeys - 1 > off + i * kBwdRows;
+            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full), ph, abort_flag, p.err, p.timeout_ns))) break;
+            tc_fence_after_sync();
+            float pr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sr[32];
+                tmem_ld32(tS + lane_sel + c * 32, sr);
+                tc_wait_ld();
+                reg_fence32(sr);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = ldg_f4(lse2 + c * 32 + e);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int col = c * 32 + e + u;
+                        float x = ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lv[u]));
+                        if (diag && col < lim) x = 0.f;
+                        pr[col] = x;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
+                tmem_st16(tS + lane_sel + c * 16, pk);
+            }
+            tc_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&ctl->p_full));
+            // dS^T = P^T (dP^T - D_i), rounded to bf16, into the [keys][rows] tile
+            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dp_full), ph, abort_flag, p.err, p.timeout_ns))) break;
+            if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->ds_empty), (w - 1) & 1u, abort_flag, p.err,
+                                                  p.timeout_ns)))
+                break;
+            tc_fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t dr[32];
+                tmem_ld32(tDP + lane_sel + c * 32, dr);
+                tc_wait_ld();
+                reg_fence32(dr);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 d4 = ldg_f4(dvec + c * 32 + e);
+                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float ds[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) ds[u] = pr[c * 32 + e + u] * (__uint_as_float(dr[e + u]) - dv4[u]);
+                    pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                    pk[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                }
+                // row t, query columns c*32 .. c*32+31: four 16-byte units of chunk c/2
+                const uint32_t rowb = sDS + (uint32_t)((c >> 1) * kChunkBytes + t * 128);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int unit = ((c & 1) * 4 + u) ^ (t & 7);
+                    st_shared_v4(rowb + unit * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&ctl->ds_full));
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ dQ, then dK and dV
+        setmaxnreg_dec<kBwdDqRegs>();
+        const int t = (warp - 8) * 32 + lane;
+        const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
+        bool ok = true;
+        for (int w = 0; w < items && ok; ++w) {
+            const int i = i0 + w / p.G;
+            const int a = g * p.G + (w - (w / p.G) * p.G);
+            const int row = i * kBwdRows + t;
+            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dq_full), w & 1u, abort_flag, p.err, p.timeout_ns))) break;
+            tc_fence_after_sync();
+            float* dst = p.dq_acc + (((size_t)b * p.Hq + a) * p.Tq + row) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tDP + lane_sel + c * 32, r);
+                tc_wait_ld();
+                reg_fence32(r);
+                if (c == D / 32 - 1) {
+                    // every column has been read: the next dP^T may overwrite them
+                    tc_fence_before_sync();
+                    mbar_arrive(smem_u32(&ctl->dq_empty));
+                }
+                if (row < p.Tq) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        red_add_v4(dst + c * 32 + e, __uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale,
+                                   __uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
+                }
+            }
+        }
+        if (ok && mbar_wait_bounded(smem_u32(&ctl->dkdv_full), 0, abort_flag, p.err, p.timeout_ns)) {
+            tc_fence_after_sync();
+            const int key = j * kBwdKeys + t;
+            const size_t orow = ((size_t)b * p.Hkv + g) * p.Tk + key;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tacc = which ? tDV : tDK;
+                const float mul = which ? 1.f : p.scale;
+                __nv_bfloat16* out = (which ? p.dv : p.dk) + orow * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tacc + lane_sel + c * 32, r);
+                    tc_wait_ld();
+                    reg_fence32(r);
+                    uint4 v4[4];
+                    uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pw[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+                    if (key < p.Tk) {
+                        uint4* d4 = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) d4[e] = v4[e];
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// D_i = <dO_i, O_i> and LSE_i * log2(e) per query row (padded to whole 128-row tiles with
+// 0 and +inf), and the fp32 dQ buffer zeroed. One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) gqa_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                           const __nv_bfloat16* __restrict__ dout,
+                                                           const float* __restrict__ lse, float* __restrict__ lse2,
+                                                           float* __restrict__ dvec, float* __restrict__ dq_acc,
+                                                           int BH, int Tq, int tq_pad) {
+    const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)BH * tq_pad) return;
+    const long long bh = gw / tq_pad;
+    const int r = (int)(gw - bh * tq_pad);
+    if (r >= Tq) {
+        if (lane == 0) {
+            lse2[gw] = INFINITY;
+            dvec[gw] = 0.f;
+        }
+        return;
+    }
+    constexpr int E = D / 32;  // elements per lane
+    const size_t base = ((size_t)bh * Tq + r) * D + lane * E;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(o[base + e]), __bfloat162float(dout[base + e]), acc);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+#pragma unroll
+    for (int e = 0; e < E; ++e) dq_acc[base + e] = 0.f;
+    if (lane == 0) {
+        dvec[gw] = acc;
+        lse2[gw] = lse[bh * Tq + r] * 1.4426950408889634f;
+    }
+}
+
+// dQ (bf16) from the fp32 buffer, 8 elements per thread.
+__global__ void __launch_bounds__(256) gqa_bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                         __nv_bfloat16* __restrict__ dq, long long n8) {
+    const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (idx >= n8) return;
+    const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * idx];
+    const float4 c = reinterpret_cast<const float4*>(dq_acc)[2 * idx + 1];
+    uint4 o;
+    o.x = pack_bf16x2(a.x, a.y);
+    o.y = pack_bf16x2(a.z, a.w);
+    o.z = pack_bf16x2(c.x, c.y);
+    o.w = pack_bf16x2(c.z, c.w);
+    reinterpret_cast<uint4*>(dq)[idx] = o;
+}
+
+}  // namespace gqa

@@ -388,6 +388,47 @@ gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, const void
     return gqa::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D) {
+    if (check_common(B, Hq, Hkv, Tq, Tk, D) != GQA_OK) return 0;
+    size_t dq_bytes, vec_bytes;
+    gqa::bwd_workspace_layout(B, Hq, Tq, D, &dq_bytes, &vec_bytes);
+    return dq_bytes + 2 * vec_bytes;
+}
+
+gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Tq, int Tk,
+                        int D, long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(lse))
+        return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    if ((long long)B * Hkv > 0x7fffffffLL || (Tk + 127) / 128 > 65535) return GQA_ERR_UNSUPPORTED;
+    size_t dq_bytes, vec_bytes;
+    gqa::bwd_workspace_layout(B, Hq, Tq, D, &dq_bytes, &vec_bytes);
+    if (!workspace || workspace_bytes < dq_bytes + 2 * vec_bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GQA_ERR_WORKSPACE;
+    gqa::BwdLaunch a{};
+    const long long q_sh = (long long)Tq * D;
+    if ((st = make_map(&a.tm_q, q, B, Hq, Tq, D, q_sh * Hq, q_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_do, dout, B, Hq, Tq, D, q_sh * Hq, q_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.o = o; a.dout = dout; a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    char* ws = static_cast<char*>(workspace);
+    a.dq_acc = reinterpret_cast<float*>(ws);
+    a.lse2 = reinterpret_cast<float*>(ws + dq_bytes);
+    a.dvec = reinterpret_cast<float*>(ws + dq_bytes + vec_bytes);
+    return gqa::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 gqa_status gqa_get_device_error(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
     uint32_t v = 0;

@@ -67,10 +67,35 @@ struct DecLaunch {
     int max_pages, page_size, num_pages, capacity;
 };
 
+// Backward (gqa_attn_bwd). The workspace holds the fp32 dQ buffer, then LSE * log2(e)
+// and <dO, O> per query row padded to whole 128-row tiles.
+struct BwdLaunch {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    int B, Hq, Hkv, Tq, Tk, D;
+    float scale;
+    const void* o;
+    const void* dout;
+    const float* lse;
+    void* dq;
+    void* dk;
+    void* dv;
+    float* dq_acc;
+    float* lse2;
+    float* dvec;
+};
+
+inline size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline void bwd_workspace_layout(int B, int Hq, int Tq, int D, size_t* dq_bytes, size_t* vec_bytes) {
+    const size_t tq_pad = (size_t)(Tq + 127) / 128 * 128;
+    *dq_bytes = round256((size_t)B * Hq * Tq * D * sizeof(float));
+    *vec_bytes = round256((size_t)B * Hq * tq_pad * sizeof(float));
+}
+
 // Each returns cudaSuccess or the launch error; nothing is synchronised.
 cudaError_t launch_fwd(const FwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_fwd_varlen(const FwdVarlenLaunch& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t stream);
 
 // Read and clear the device error word of the current device (after a stream sync).

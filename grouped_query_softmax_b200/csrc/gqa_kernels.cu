@@ -5,6 +5,7 @@
 
 #include <algorithm>
 
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "gqa_internal.h"
@@ -176,6 +177,52 @@ cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream) {
     if (a.seqlens != nullptr)
         return a.D == 128 ? launch_decode_d<128, true>(a, stream) : launch_decode_d<64, true>(a, stream);
     return a.D == 128 ? launch_decode_d<128, false>(a, stream) : launch_decode_d<64, false>(a, stream);
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
+    BwdParams p{};
+    p.B = a.B;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.Tq = a.Tq;
+    p.Tk = a.Tk;
+    p.G = a.Hq / a.Hkv;
+    p.n_qt = (a.Tq + kBwdRows - 1) / kBwdRows;
+    p.tq_pad = p.n_qt * kBwdRows;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.lse2 = a.lse2;
+    p.dvec = a.dvec;
+    p.dq_acc = a.dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(a.dk);
+    p.dv = static_cast<__nv_bfloat16*>(a.dv);
+    p.err = device_error_ptr();
+    p.timeout_ns = kWaitTimeoutNs;
+    if (!p.err) return cudaErrorUnknown;
+    const int smem = BwdSmem<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(gqa_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, gqa_bwd_sm100_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split needs it
+    const long long rows = (long long)a.B * a.Hq * p.tq_pad;
+    gqa_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.lse2, a.dvec,
+        a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 grid((unsigned)(a.B * a.Hkv), (unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys));
+    gqa_bwd_sm100_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long n8 = (long long)a.B * a.Hq * a.Tq * a.D / 8;
+    gqa_bwd_dq_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.dq),
+                                                                        n8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const BwdLaunch& a, cudaStream_t stream) {
+    return a.D == 128 ? launch_bwd_d<128>(a, stream) : launch_bwd_d<64>(a, stream);
 }
 
 // One CTA, one thread: wait on an mbarrier that never completes, bounded by

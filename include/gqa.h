@@ -271,6 +271,34 @@ GQA_API gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, co
                                           float softmax_scale, int window, int num_splits,
                                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Backward pass: dQ, dK and dV of gqa_attn_fwd for an output gradient dO (training).
+ * With P the softmax weights of each row over its visible keys and D_i = <dO_i, O_i>:
+ *   dV_j = sum_i P_ij dO_i,   dS_ij = P_ij (<dO_i, v_j> - D_i),
+ *   dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i,
+ * the derivative of the o_a definition ("注意力家族", section 统一记号); a KV head's dK and
+ * dV sum over the H_q/H_kv query heads that read it. As in the FlashAttention backward
+ * ("长上下文与高效注意力：研究账本", section FlashAttention: the backward recomputes, which
+ * adds FLOPs), P is recomputed from q, k and the forward's log-sum-exp.
+ *
+ *   q, o, dout  bf16 [B, Hq, Tq, D], contiguous: the forward's inputs and output, and dO.
+ *   k, v        as for gqa_attn_fwd (first Tk rows, free batch/head strides).
+ *   lse         fp32 [B, Hq, Tq]: the natural-log LSE gqa_attn_fwd returned for o.
+ *   dq          bf16 [B, Hq, Tq, D], contiguous; written.
+ *   dk, dv      bf16 [B, Hkv, Tk, D], contiguous; written (the gradient of the [:Tk] slice).
+ *   workspace   device, >= gqa_attn_bwd_workspace_bytes(...) bytes, 256-byte aligned
+ *               (an fp32 copy of dQ plus two fp32 values per query row); contents on
+ *               entry ignored; not shared by calls that can overlap on the GPU.
+ * Causal only (no window). dQ is accumulated with fp32 atomic additions, so its last
+ * bits can differ from run to run; dK and dV are deterministic.
+ */
+GQA_API size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D);
+GQA_API gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb,
+                                long long k_sh, long long v_sb, long long v_sh, float softmax_scale,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* A static, human-readable name for a status code. */
 GQA_API const char* gqa_status_string(gqa_status s);
 

@@ -180,3 +180,26 @@ def test_varlen_decode_split_planning(gqa):
             gqa.gqa_attn_decode_ex_num_splits(4, 8, 2, 1, 4096, 128, 0, s)
     assert gqa.gqa_attn_decode_varlen_workspace_bytes(64, 32, 8, 1, 32768, 128, 0, 1) == 0
     assert gqa.gqa_attn_decode_varlen_workspace_bytes(64, 32, 8, 17, 32768, 128, 0, 0) == 0  # Tq > 16
+
+
+def bwd(gqa, **kw):
+    a = dict(q=P, k=P, v=P, o=P, dout=P, lse=P, dq=P, dk=P, dv=P, B=1, Hq=4, Hkv=2, Tq=8, Tk=8, D=64,
+             k_sb=2 * 8 * 64, k_sh=8 * 64, v_sb=2 * 8 * 64, v_sh=8 * 64, softmax_scale=0.0,
+             workspace=P, workspace_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_bwd(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), 1), (dict(Tq=9), 1), (dict(dk=None), 1), (dict(lse=P + 4), 1), (dict(D=96), 2),
+    (dict(k_sh=8 * 64 + 4), 1), (dict(workspace=None), 3), (dict(workspace_bytes=16), 3),
+    (dict(workspace=P + 64), 3),
+])
+def test_bwd_rejects_bad_arguments(gqa, kw, status):
+    assert bwd(gqa, **kw) == status
+
+
+def test_bwd_workspace_size(gqa):
+    # fp32 dQ [B,Hq,Tq,D] + two fp32 values per row padded to 128-row tiles, each 256-aligned
+    assert gqa.gqa_attn_bwd_workspace_bytes(1, 4, 2, 8, 8, 64) == 8192 + 2 * 2048
+    assert gqa.gqa_attn_bwd_workspace_bytes(1, 4, 2, 9, 8, 64) == 0
