@@ -286,6 +286,36 @@ def measure_decode(w, steps, warmup, world, dev, e2e_steps):
     return res
 
 
+def bwd_flops(w) -> float:
+    """Backward FLOPs: five products per visible pair (S recomputed, dP, dV, dK, dQ), each
+    2 * D per pair and query head: 10 * D * Hq * B * pairs = 2.5x the forward's."""
+    return 10.0 * w.D * w.Hq * w.B * visible_pairs(w.Tq, w.Tk, w.window)
+
+
+def measure_bwd(w, steps, warmup, world, dev):
+    """gqa_attn_bwd on a dense workload: prep + attention backward + dQ rounding per step;
+    the forward's output and log-sum-exp are computed once, before the timed region."""
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, k, v = w.make()
+    do = w.make_dout()
+    qd, kd, vd, dod = (to_device(x, dev) for x in (q, k, v, do))
+    o, lse = gqa.attn_fwd(qd, kd, vd, return_lse=True)
+    dq = torch.empty_like(qd)
+    dk = torch.empty_like(kd)
+    dv = torch.empty_like(vd)
+    ws = torch.empty(gqa.gqa_attn_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.Tq, w.Tk, w.D), dtype=torch.uint8,
+                     device=dev)
+    fn = lambda: gqa.attn_bwd(qd, kd, vd, o, dod, lse, dq=dq, dk=dk, dv=dv, workspace=ws)
+    ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after backward timing: {gqa.gqa_status_string(st)}")
+    del qd, kd, vd, dod, o, lse, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return {"ms_total": ms, "t0": t0, "t1": t1, "launches": 3 * steps}
+
+
 def varlen_flops(w) -> float:
     """4 * D * Hq * sum over sequences of their causal-visible pairs."""
     lq, lk = w.lengths()
@@ -433,6 +463,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the sliding-window, decode-chunk and variable-length measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--backward", action="store_true",
+                    help="measure only the backward pass of the main (dense) workload, e.g. for profiling")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--batch", type=int, default=0,
@@ -496,6 +528,35 @@ def reference_arm(args, rank, world):
                              "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def backward_main(args, rank, world, local, dev, peaks, peak_src, w):
+    """The backward pass of a dense workload as the main line (profiling and focused runs)."""
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local])
+    sampler.start()
+    time.sleep(0.2)
+    r = measure_bwd(w, args.steps, args.warmup, world, dev)
+    ms_step = r["ms_total"] / args.steps
+    achieved = bwd_flops(w) / (ms_step * 1e-3) / 1e12
+    clocks = sampler.summary(r["t0"], r["t1"])
+    sampler.stop()
+    line = {"metric": "GQA attn backward TFLOP/s on 1 B200, % of roofline", "value": world * achieved,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, {"pass": "backward (dQ, dK, dV)", "l2": "inputs larger than L2 (no flush)",
+                                          "parallelism": f"dp{world} (independent problems per rank)"}),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": load_traffic("gqa_bwd_sm100_kernel", w.name),
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "kernel": "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"},
+            "gpu_launches": r["launches"], "clocks": clocks}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def varlen_main(args, rank, world, local, dev, peaks, peak_src):
@@ -573,6 +634,8 @@ def main(argv=None):
     if args.batch > 0:
         import dataclasses
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name} (batch {args.batch})")
+    if args.backward:
+        return backward_main(args, rank, world, local, dev, peaks, peak_src, w)
     gpu_id = None
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -689,6 +752,20 @@ def main(argv=None):
                              "traffic": load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
                 "gpu_launches": rv["launches"]}
+        # backward (training) on the headline workload
+        nsb = max(10, args.steps // 4)
+        rb = measure_bwd(w, nsb, max(3, args.warmup), world, dev)
+        msb = rb["ms_total"] / nsb
+        achb = bwd_flops(w) / (msb * 1e-3) / 1e12
+        line["backward"] = {
+            "metric": "TFLOP/s (10 * D * Hq * B * causal-visible pairs: S, dP, dV, dK, dQ)", "value": world * achb,
+            "unit": "TFLOP/s", "ms_per_step": msb, "config": workload_config(w),
+            "roofline": {"bound": "tensor", "achieved": achb, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achb / peaks["bf16_tflops"],
+                         "traffic": load_traffic("gqa_bwd_sm100_kernel", w.name),
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "kernel": "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"},
+            "gpu_launches": rb["launches"]}
         wp = gi.VARLEN_WORKLOADS["paged_decode"]
         nsp = max(3, args.steps // 20)
         rp = measure_paged_decode(wp, nsp, max(3, args.warmup), world, dev)

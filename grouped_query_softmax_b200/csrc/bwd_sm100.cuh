@@ -20,7 +20,8 @@
 //   dS^T = P^T (dP^T - D_i)  -> shared memory, bf16, [keys][rows]
 //   dK  += dS^T Q_i       (A = dS^T, K-major)
 //   dQ_i = dS K_j         (A = the same buffer read M-major), added into an fp32 dQ buffer
-// Warps: 0 TMA producer (K_j, V_j once; Q_i and dO_i through a 2-slot ring), 1 tcgen05
+// Warps: 0 TMA producer (K_j, V_j once; Q_i and dO_i through a 2-slot ring; each step's
+// LSE and D vectors by bulk copy), 1 tcgen05
 // issuer, 2 TMEM allocation, 4-7 the P / dS warpgroup (thread t owns key row t and keeps
 // its 128 probabilities in registers), 8-11 the dQ warpgroup (thread t owns query row t of
 // the dQ tile; adds it to the fp32 buffer with vector reductions) and, at the end, the dK
@@ -68,11 +69,14 @@ struct BwdSmem {
     static constexpr int kSlotBytes = 2 * kTileBytes;
     static constexpr int kDsOff = kRingOff + 2 * kSlotBytes;  // dS^T [128 keys][128 rows] bf16
     static constexpr int kDsBytes = 2 * kChunkBytes;
-    static constexpr int kCtlOff = kDsOff + kDsBytes;
+    static constexpr int kLseOff = kDsOff + kDsBytes;       // LSE_i log2(e) of the current step
+    static constexpr int kDvecOff = kLseOff + 4 * kBwdRows;  // D_i of the current step
+    static constexpr int kCtlOff = kDvecOff + 4 * kBwdRows;
     struct Ctl {
         uint64_t kv_full;
         uint64_t qdo_full[2];
         uint64_t qdo_empty[2];
+        uint64_t lse_full, dvec_full;
         uint64_t s_full, p_full, dp_full, ds_full, ds_empty, dq_full, dq_empty, dkdv_full;
         uint64_t drain;
         uint32_t tmem_base;
@@ -94,10 +98,6 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                  : "memory");
 }
 
-__device__ __forceinline__ float4 ldg_f4(const float* p) {
-    return __ldg(reinterpret_cast<const float4*>(p));
-}
-
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gqa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -117,15 +117,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t sV = sbase + L::kVOff;
     const uint32_t sRing = sbase + L::kRingOff;
     const uint32_t sDS = sbase + L::kDsOff;
+    const uint32_t sLse = sbase + L::kLseOff;
+    const uint32_t sDvec = sbase + L::kDvecOff;
+    const float* lse_s = reinterpret_cast<const float*>(smem + L::kLseOff);
+    const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvecOff);
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtlOff);
     volatile uint32_t* abort_flag = &ctl->abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bg = blockIdx.x;  // b * Hkv + g
+    // Key blocks of one (b, g) are launched together: they all add into the same dQ rows,
+    // which then stay in L2 while they run. Within a (b, g), low j first (most work).
+    const int j = blockIdx.x;
+    const int bg = blockIdx.y;  // b * Hkv + g
     const int b = bg / p.Hkv;
     const int g = bg - b * p.Hkv;
-    const int j = blockIdx.y;   // key block; low j first (they have the most work)
     const int off = p.Tk - p.Tq;
     const int i0 = bwd_first_tile(j, p.Tq, p.Tk);
     const int items = p.G * (p.n_qt - i0);  // (query tile, head) steps, tile-major
@@ -136,6 +142,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(smem_u32(&ctl->qdo_full[s]), 1);
             mbar_init(smem_u32(&ctl->qdo_empty[s]), 1);
         }
+        mbar_init(smem_u32(&ctl->lse_full), 1);
+        mbar_init(smem_u32(&ctl->dvec_full), 1);
         mbar_init(smem_u32(&ctl->s_full), 1);
         mbar_init(smem_u32(&ctl->p_full), 128);
         mbar_init(smem_u32(&ctl->dp_full), 1);
@@ -179,6 +187,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_4d(sV + c * kChunkBytes, &tm_v, kvbar, c * 64, j * kBwdKeys, g, b);
             }
             uint32_t issued[2] = {0u, 0u};
+            uint32_t vec_issued = 0;  // LSE (and D) vectors copied
+            const uint32_t lbar = smem_u32(&ctl->lse_full), dbar = smem_u32(&ctl->dvec_full);
             for (int w = 0; w < items && ok; ++w) {
                 const int slot = w & 1;
                 const int i = i0 + w / p.G;
@@ -194,11 +204,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tma_load_4d(sQ + kTileBytes + c * kChunkBytes, &tm_do, fbar, c * 64, i * kBwdRows, a, b);
                 }
                 ++issued[slot];
+                // the step's LSE and D vectors (one slot each): LSE once the previous step's P
+                // is done with it, D once the previous step's dS is
+                const size_t vrow = ((size_t)b * p.Hq + a) * p.tq_pad + (size_t)i * kBwdRows;
+                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->p_full), (w - 1) & 1u, abort_flag, p.err,
+                                                      p.timeout_ns)))
+                    break;
+                mbar_arrive_expect_tx(lbar, 4 * kBwdRows);
+                bulk_load(sLse, p.lse2 + vrow, 4 * kBwdRows, lbar);
+                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), (w - 1) & 1u, abort_flag, p.err,
+                                                      p.timeout_ns))) {
+                    ++vec_issued;  // the LSE copy is in flight
+                    break;
+                }
+                mbar_arrive_expect_tx(dbar, 4 * kBwdRows);
+                bulk_load(sDvec, p.dvec + vrow, 4 * kBwdRows, dbar);
+                ++vec_issued;
             }
             if (*abort_flag) {
                 mbar_wait_drain(kvbar, 0, p.timeout_ns);
                 for (int s = 0; s < 2; ++s)
                     if (issued[s]) mbar_wait_drain(smem_u32(&ctl->qdo_full[s]), (issued[s] - 1u) & 1u, p.timeout_ns);
+                if (vec_issued) {
+                    mbar_wait_drain(lbar, (vec_issued - 1u) & 1u, p.timeout_ns);
+                    mbar_wait_drain(dbar, (vec_issued - 1u) & 1u, p.timeout_ns);
+                }
             }
         }
     } else if (warp == 1) {
@@ -212,28 +242,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t dK_nmaj = umma_desc_sw128(sK, kChunkBytes, 1024);
             const uint64_t dS_kmaj = umma_desc_sw128(sDS, 16, 1024);
             const uint64_t dS_mmaj = umma_desc_sw128(sDS, kChunkBytes, 1024);
-            bool ok = mbar_wait_bounded(smem_u32(&ctl->kv_full), 0, abort_flag, p.err, p.timeout_ns);
-            tc_fence_after_sync();
-            for (int w = 0; w < items && ok; ++w) {
-                const int slot = w & 1;
-                const uint32_t ph = w & 1;
-                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->qdo_full[slot]), (w >> 1) & 1u, abort_flag, p.err,
-                                             p.timeout_ns)))
-                    break;
+            // S^T = K_j Q_i^T of step w: M = 128 keys, N = 128 rows, K = D in steps of 16
+            auto issue_s = [&](int w) -> bool {
+                if (!mbar_wait_bounded(smem_u32(&ctl->qdo_full[w & 1]), (w >> 1) & 1u, abort_flag, p.err,
+                                       p.timeout_ns))
+                    return false;
                 tc_fence_after_sync();
-                const uint32_t sQ = sRing + slot * L::kSlotBytes;
-                const uint32_t sDO = sQ + kTileBytes;
-                const uint64_t dQ_kmaj = umma_desc_sw128(sQ, 16, 1024);
-                const uint64_t dDO_kmaj = umma_desc_sw128(sDO, 16, 1024);
-                const uint64_t dQ_nmaj = umma_desc_sw128(sQ, kChunkBytes, 1024);
-                const uint64_t dDO_nmaj = umma_desc_sw128(sDO, kChunkBytes, 1024);
-                // S^T = K_j Q_i^T: M = 128 keys, N = 128 rows, K = D in steps of 16
+                const uint64_t dQ_kmaj = umma_desc_sw128(sRing + (w & 1) * L::kSlotBytes, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
                     tc_mma_ss(tS, dK_kmaj + ko, dQ_kmaj + ko, idesc_t, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(&ctl->s_full));
+                return true;
+            };
+            bool ok = mbar_wait_bounded(smem_u32(&ctl->kv_full), 0, abort_flag, p.err, p.timeout_ns);
+            tc_fence_after_sync();
+            if (ok && items > 0) ok = issue_s(0);
+            for (int w = 0; w < items && ok; ++w) {
+                const int slot = w & 1;
+                const uint32_t ph = w & 1;
+                const uint32_t sQ = sRing + slot * L::kSlotBytes;
+                const uint32_t sDO = sQ + kTileBytes;
+                const uint64_t dDO_kmaj = umma_desc_sw128(sDO, 16, 1024);
+                const uint64_t dQ_nmaj = umma_desc_sw128(sQ, kChunkBytes, 1024);
+                const uint64_t dDO_nmaj = umma_desc_sw128(sDO, kChunkBytes, 1024);
                 // dP^T = V_j dO_i^T into the dQ columns, once the previous dQ has been read
                 if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->dq_empty), (w - 1) & 1u, abort_flag, p.err,
                                                       p.timeout_ns)))
@@ -252,6 +286,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int kk = 0; kk < kBwdRows / 16; ++kk)
                     tc_mma_ts(tDV, tS + kk * 8, dDO_nmaj + (uint64_t)((kk * 2048) >> 4), idesc_kv,
                               (w > 0 || kk > 0) ? 1u : 0u);
+                // the next step's S^T now: it runs while this step's dS is formed (the tensor
+                // pipe executes in order, so dV has read P^T before S^T overwrites it)
+                if (w + 1 < items && !(ok = issue_s(w + 1))) break;
                 // dK += dS^T Q_i and dQ_i = dS K_j, once dS^T is in shared memory
                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), ph, abort_flag, p.err, p.timeout_ns))) break;
                 tc_fence_after_sync();
@@ -286,12 +323,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t ph = w & 1;
             const int i = i0 + w / p.G;
             const int a = g * p.G + (w - (w / p.G) * p.G);
-            const size_t vrow = ((size_t)b * p.Hq + a) * p.tq_pad + (size_t)i * kBwdRows;
-            const float* lse2 = p.lse2 + vrow;
-            const float* dvec = p.dvec + vrow;
+            (void)a;
             // column c (query row i*128 + c) sees this key iff c >= lim
             const int lim = kabs - (off + i * kBwdRows);
             const bool diag = j * kBwdKeys + kBwdKeys - 1 > off + i * kBwdRows;
+            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->lse_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             tc_fence_after_sync();
             float pr[128];
@@ -304,7 +340,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = ldg_f4(lse2 + c * 32 + e);
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + e);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -323,6 +359,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_arrive(smem_u32(&ctl->p_full));
             // dS^T = P^T (dP^T - D_i), rounded to bf16, into the [keys][rows] tile
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dp_full), ph, abort_flag, p.err, p.timeout_ns))) break;
+            if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dvec_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->ds_empty), (w - 1) & 1u, abort_flag, p.err,
                                                   p.timeout_ns)))
                 break;
@@ -336,7 +373,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 d4 = ldg_f4(dvec + c * 32 + e);
+                    const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + e);
                     const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
                     float ds[4];
 #pragma unroll

@@ -407,7 +407,7 @@ gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
     if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
     if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
-    if ((long long)B * Hkv > 0x7fffffffLL || (Tk + 127) / 128 > 65535) return GQA_ERR_UNSUPPORTED;
+    if ((long long)B * Hkv > 65535 || (Tk + 127) / 128 > 0x7fffffff) return GQA_ERR_UNSUPPORTED;  // grid y, x
     size_t dq_bytes, vec_bytes;
     gqa::bwd_workspace_layout(B, Hq, Tq, D, &dq_bytes, &vec_bytes);
     if (!workspace || workspace_bytes < dq_bytes + 2 * vec_bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))

@@ -212,7 +212,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.lse2, a.dvec,
         a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const dim3 grid((unsigned)(a.B * a.Hkv), (unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys));
+    const dim3 grid((unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys), (unsigned)(a.B * a.Hkv));
     gqa_bwd_sm100_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long n8 = (long long)a.B * a.Hq * a.Tq * a.D / 8;
