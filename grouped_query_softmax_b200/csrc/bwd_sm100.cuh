@@ -20,12 +20,13 @@
 //   dS^T = P^T (dP^T - D_i)  -> shared memory, bf16, [keys][rows]
 //   dK  += dS^T Q_i       (A = dS^T, K-major)
 //   dQ_i = dS K_j         (A = the same buffer read M-major), added into an fp32 dQ buffer
-// Warps: 0 TMA producer (K_j, V_j once; Q_i and dO_i through a 2-slot ring; each step's
-// LSE and D vectors by bulk copy), 1 tcgen05
-// issuer, 2 TMEM allocation, 4-7 the P / dS warpgroup (thread t owns key row t and keeps
-// its 128 probabilities in registers), 8-11 the dQ warpgroup (thread t owns query row t of
-// the dQ tile; adds it to the fp32 buffer with vector reductions) and, at the end, the dK
-// and dV epilogue. TMEM (512 columns at D = 128): S^T | dP^T, later dQ | dV | dK.
+// Warps: 0 TMA producer (K_j, V_j once; Q_i through a 2-slot ring, dO_i through one slot
+// released right after dV; each step's LSE and D vectors by bulk copy), 1 tcgen05 issuer,
+// 2 TMEM allocation, 4-7 the P / dS warpgroup (thread t owns key row t and keeps its 128
+// probabilities in registers), 8-11 the dQ warpgroup (thread t owns query row t of the dQ
+// tile; it stages 64 columns at a time in shared memory and one thread adds them to the
+// fp32 buffer with a TMA bulk reduction) and, at the end, the dK and dV epilogue.
+// TMEM (512 columns at D = 128): S^T | dP^T, later dQ | dV | dK.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -65,19 +66,23 @@ struct BwdSmem {
     static constexpr int kTileBytes = kChunks * kChunkBytes;  // one [128][D] bf16 tile
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kTileBytes;
-    static constexpr int kRingOff = 2 * kTileBytes;        // 2 slots of (Q_i, dO_i)
-    static constexpr int kSlotBytes = 2 * kTileBytes;
-    static constexpr int kDsOff = kRingOff + 2 * kSlotBytes;  // dS^T [128 keys][128 rows] bf16
+    static constexpr int kQOff = 2 * kTileBytes;           // 2 slots of Q_i
+    static constexpr int kDoOff = 4 * kTileBytes;          // 1 slot of dO_i
+    static constexpr int kDsOff = 5 * kTileBytes;          // dS^T [128 keys][128 rows] bf16
     static constexpr int kDsBytes = 2 * kChunkBytes;
-    static constexpr int kLseOff = kDsOff + kDsBytes;       // LSE_i log2(e) of the current step
+    static constexpr int kStageOff = kDsOff + kDsBytes;    // dQ staging: [128 rows][64 fp32], two boxes
+    static constexpr int kStageBytes = 2 * kChunkBytes;    // of [128][32] in the 128-byte swizzle
+    static constexpr int kLseOff = kStageOff + kStageBytes;  // LSE_i log2(e) of the current step
     static constexpr int kDvecOff = kLseOff + 4 * kBwdRows;  // D_i of the current step
     static constexpr int kCtlOff = kDvecOff + 4 * kBwdRows;
     struct Ctl {
         uint64_t kv_full;
-        uint64_t qdo_full[2];
-        uint64_t qdo_empty[2];
+        uint64_t q_full[2];
+        uint64_t q_empty[2];
+        uint64_t do_full, do_empty;
         uint64_t lse_full, dvec_full;
         uint64_t s_full, p_full, dp_full, ds_full, ds_empty, dq_full, dq_empty, dkdv_full;
+        uint64_t stage_full, stage_free;
         uint64_t drain;
         uint32_t tmem_base;
         uint32_t abort;
@@ -92,17 +97,11 @@ __device__ __forceinline__ int bwd_first_tile(int j, int Tq, int Tk) {
     return r > 0 ? r / kBwdRows : 0;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gqa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                         const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using L = BwdSmem<D>;
     using Ctl = typename L::Ctl;
     constexpr int kTileBytes = L::kTileBytes;
@@ -115,8 +114,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t sbase = raw_addr + pad;
     const uint32_t sK = sbase + L::kKOff;
     const uint32_t sV = sbase + L::kVOff;
-    const uint32_t sRing = sbase + L::kRingOff;
+    const uint32_t sQ0 = sbase + L::kQOff;
+    const uint32_t sDO = sbase + L::kDoOff;
     const uint32_t sDS = sbase + L::kDsOff;
+    const uint32_t sStage = sbase + L::kStageOff;
     const uint32_t sLse = sbase + L::kLseOff;
     const uint32_t sDvec = sbase + L::kDvecOff;
     const float* lse_s = reinterpret_cast<const float*>(smem + L::kLseOff);
@@ -139,9 +140,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl->kv_full), 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&ctl->qdo_full[s]), 1);
-            mbar_init(smem_u32(&ctl->qdo_empty[s]), 1);
+            mbar_init(smem_u32(&ctl->q_full[s]), 1);
+            mbar_init(smem_u32(&ctl->q_empty[s]), 1);
         }
+        mbar_init(smem_u32(&ctl->do_full), 1);
+        mbar_init(smem_u32(&ctl->do_empty), 1);
+        mbar_init(smem_u32(&ctl->stage_full), 128);
+        mbar_init(smem_u32(&ctl->stage_free), 1);
         mbar_init(smem_u32(&ctl->lse_full), 1);
         mbar_init(smem_u32(&ctl->dvec_full), 1);
         mbar_init(smem_u32(&ctl->s_full), 1);
@@ -165,6 +170,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
+        prefetch_tensormap(&tm_dq);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -186,49 +192,53 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_4d(sK + c * kChunkBytes, &tm_k, kvbar, c * 64, j * kBwdKeys, g, b);
                 tma_load_4d(sV + c * kChunkBytes, &tm_v, kvbar, c * 64, j * kBwdKeys, g, b);
             }
-            uint32_t issued[2] = {0u, 0u};
-            uint32_t vec_issued = 0;  // LSE (and D) vectors copied
+            uint32_t q_issued[2] = {0u, 0u};
+            uint32_t lse_issued = 0, do_issued = 0, dvec_issued = 0;
             const uint32_t lbar = smem_u32(&ctl->lse_full), dbar = smem_u32(&ctl->dvec_full);
+            const uint32_t obar = smem_u32(&ctl->do_full);
             for (int w = 0; w < items && ok; ++w) {
                 const int slot = w & 1;
                 const int i = i0 + w / p.G;
                 const int a = g * p.G + (w - (w / p.G) * p.G);
-                if (w >= 2 && !(ok = mbar_wait_bounded(smem_u32(&ctl->qdo_empty[slot]), ((w >> 1) - 1) & 1u,
+                // Q_i: two slots (the next step's S^T is issued while this step still needs Q_i)
+                if (w >= 2 && !(ok = mbar_wait_bounded(smem_u32(&ctl->q_empty[slot]), ((w >> 1) - 1) & 1u,
                                                        abort_flag, p.err, p.timeout_ns)))
                     break;
-                const uint32_t fbar = smem_u32(&ctl->qdo_full[slot]);
-                const uint32_t sQ = sRing + slot * L::kSlotBytes;
-                mbar_arrive_expect_tx(fbar, 2 * kTileBytes);
-                for (int c = 0; c < L::kChunks; ++c) {
-                    tma_load_4d(sQ + c * kChunkBytes, &tm_q, fbar, c * 64, i * kBwdRows, a, b);
-                    tma_load_4d(sQ + kTileBytes + c * kChunkBytes, &tm_do, fbar, c * 64, i * kBwdRows, a, b);
-                }
-                ++issued[slot];
-                // the step's LSE and D vectors (one slot each): LSE once the previous step's P
-                // is done with it, D once the previous step's dS is
+                const uint32_t qbar = smem_u32(&ctl->q_full[slot]);
+                mbar_arrive_expect_tx(qbar, kTileBytes);
+                for (int c = 0; c < L::kChunks; ++c)
+                    tma_load_4d(sQ0 + slot * kTileBytes + c * kChunkBytes, &tm_q, qbar, c * 64, i * kBwdRows, a, b);
+                ++q_issued[slot];
+                // LSE once the previous step's P is done with it, dO once the previous dV has
+                // read it, D once the previous step's dS is done (one slot each)
                 const size_t vrow = ((size_t)b * p.Hq + a) * p.tq_pad + (size_t)i * kBwdRows;
                 if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->p_full), (w - 1) & 1u, abort_flag, p.err,
                                                       p.timeout_ns)))
                     break;
                 mbar_arrive_expect_tx(lbar, 4 * kBwdRows);
                 bulk_load(sLse, p.lse2 + vrow, 4 * kBwdRows, lbar);
-                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), (w - 1) & 1u, abort_flag, p.err,
-                                                      p.timeout_ns))) {
-                    ++vec_issued;  // the LSE copy is in flight
+                ++lse_issued;
+                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->do_empty), (w - 1) & 1u, abort_flag, p.err,
+                                                      p.timeout_ns)))
                     break;
-                }
+                mbar_arrive_expect_tx(obar, kTileBytes);
+                for (int c = 0; c < L::kChunks; ++c)
+                    tma_load_4d(sDO + c * kChunkBytes, &tm_do, obar, c * 64, i * kBwdRows, a, b);
+                ++do_issued;
+                if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), (w - 1) & 1u, abort_flag, p.err,
+                                                      p.timeout_ns)))
+                    break;
                 mbar_arrive_expect_tx(dbar, 4 * kBwdRows);
                 bulk_load(sDvec, p.dvec + vrow, 4 * kBwdRows, dbar);
-                ++vec_issued;
+                ++dvec_issued;
             }
             if (*abort_flag) {
                 mbar_wait_drain(kvbar, 0, p.timeout_ns);
                 for (int s = 0; s < 2; ++s)
-                    if (issued[s]) mbar_wait_drain(smem_u32(&ctl->qdo_full[s]), (issued[s] - 1u) & 1u, p.timeout_ns);
-                if (vec_issued) {
-                    mbar_wait_drain(lbar, (vec_issued - 1u) & 1u, p.timeout_ns);
-                    mbar_wait_drain(dbar, (vec_issued - 1u) & 1u, p.timeout_ns);
-                }
+                    if (q_issued[s]) mbar_wait_drain(smem_u32(&ctl->q_full[s]), (q_issued[s] - 1u) & 1u, p.timeout_ns);
+                if (lse_issued) mbar_wait_drain(lbar, (lse_issued - 1u) & 1u, p.timeout_ns);
+                if (do_issued) mbar_wait_drain(obar, (do_issued - 1u) & 1u, p.timeout_ns);
+                if (dvec_issued) mbar_wait_drain(dbar, (dvec_issued - 1u) & 1u, p.timeout_ns);
             }
         }
     } else if (warp == 1) {
@@ -244,11 +254,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t dS_mmaj = umma_desc_sw128(sDS, kChunkBytes, 1024);
             // S^T = K_j Q_i^T of step w: M = 128 keys, N = 128 rows, K = D in steps of 16
             auto issue_s = [&](int w) -> bool {
-                if (!mbar_wait_bounded(smem_u32(&ctl->qdo_full[w & 1]), (w >> 1) & 1u, abort_flag, p.err,
+                if (!mbar_wait_bounded(smem_u32(&ctl->q_full[w & 1]), (w >> 1) & 1u, abort_flag, p.err,
                                        p.timeout_ns))
                     return false;
                 tc_fence_after_sync();
-                const uint64_t dQ_kmaj = umma_desc_sw128(sRing + (w & 1) * L::kSlotBytes, 16, 1024);
+                const uint64_t dQ_kmaj = umma_desc_sw128(sQ0 + (w & 1) * kTileBytes, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
@@ -260,15 +270,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool ok = mbar_wait_bounded(smem_u32(&ctl->kv_full), 0, abort_flag, p.err, p.timeout_ns);
             tc_fence_after_sync();
             if (ok && items > 0) ok = issue_s(0);
+            const uint64_t dDO_kmaj = umma_desc_sw128(sDO, 16, 1024);
+            const uint64_t dDO_nmaj = umma_desc_sw128(sDO, kChunkBytes, 1024);
             for (int w = 0; w < items && ok; ++w) {
                 const int slot = w & 1;
                 const uint32_t ph = w & 1;
-                const uint32_t sQ = sRing + slot * L::kSlotBytes;
-                const uint32_t sDO = sQ + kTileBytes;
-                const uint64_t dDO_kmaj = umma_desc_sw128(sDO, 16, 1024);
-                const uint64_t dQ_nmaj = umma_desc_sw128(sQ, kChunkBytes, 1024);
-                const uint64_t dDO_nmaj = umma_desc_sw128(sDO, kChunkBytes, 1024);
-                // dP^T = V_j dO_i^T into the dQ columns, once the previous dQ has been read
+                const uint64_t dQ_nmaj = umma_desc_sw128(sQ0 + slot * kTileBytes, kChunkBytes, 1024);
+                // dP^T = V_j dO_i^T into the dQ columns, once dO_i has landed and the previous
+                // dQ has been read
+                if (!(ok = mbar_wait_bounded(smem_u32(&ctl->do_full), ph, abort_flag, p.err, p.timeout_ns))) break;
                 if (w > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->dq_empty), (w - 1) & 1u, abort_flag, p.err,
                                                       p.timeout_ns)))
                     break;
@@ -286,6 +296,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int kk = 0; kk < kBwdRows / 16; ++kk)
                     tc_mma_ts(tDV, tS + kk * 8, dDO_nmaj + (uint64_t)((kk * 2048) >> 4), idesc_kv,
                               (w > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(smem_u32(&ctl->do_empty));  // dV is dO_i's last reader
                 // the next step's S^T now: it runs while this step's dS is formed (the tensor
                 // pipe executes in order, so dV has read P^T before S^T overwrites it)
                 if (w + 1 < items && !(ok = issue_s(w + 1))) break;
@@ -304,7 +315,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                               idesc_q, kk > 0 ? 1u : 0u);
                 tc_commit(smem_u32(&ctl->dq_full));
                 tc_commit(smem_u32(&ctl->ds_empty));
-                tc_commit(smem_u32(&ctl->qdo_empty[slot]));
+                tc_commit(smem_u32(&ctl->q_empty[slot]));
             }
             if (ok) tc_commit(smem_u32(&ctl->dkdv_full));
             if (*abort_flag) {
@@ -399,32 +410,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int t = (warp - 8) * 32 + lane;
         const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
+        uint32_t rounds = 0;  // staging rounds so far (64 dQ columns each)
         for (int w = 0; w < items && ok; ++w) {
             const int i = i0 + w / p.G;
             const int a = g * p.G + (w - (w / p.G) * p.G);
-            const int row = i * kBwdRows + t;
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dq_full), w & 1u, abort_flag, p.err, p.timeout_ns))) break;
             tc_fence_after_sync();
-            float* dst = p.dq_acc + (((size_t)b * p.Hq + a) * p.Tq + row) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tDP + lane_sel + c * 32, r);
+            for (int h = 0; h < D / 64 && ok; ++h, ++rounds) {
+                // the previous round's bulk reduction has finished reading the staging tile
+                if (rounds > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->stage_free), (rounds - 1) & 1u, abort_flag,
+                                                           p.err, p.timeout_ns)))
+                    break;
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tDP + lane_sel + h * 64, r0);
+                tmem_ld32(tDP + lane_sel + h * 64 + 32, r1);
                 tc_wait_ld();
-                reg_fence32(r);
-                if (c == D / 32 - 1) {
-                    // every column has been read: the next dP^T may overwrite them
+                reg_fence32(r0);
+                reg_fence32(r1);
+                if (h == D / 64 - 1) {
+                    // every dQ column has been read: the next dP^T may overwrite them
                     tc_fence_before_sync();
                     mbar_arrive(smem_u32(&ctl->dq_empty));
                 }
-                if (row < p.Tq) {
+                // row t of two [128][32] fp32 boxes, 16-byte units in the 128-byte swizzle
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        red_add_v4(dst + c * 32 + e, __uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale,
-                                   __uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
+                for (int bx = 0; bx < 2; ++bx) {
+                    const uint32_t* rr = bx ? r1 : r0;
+                    const uint32_t rowb = sStage + bx * kChunkBytes + t * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        st_shared_v4(rowb + ((u ^ (t & 7)) * 16),
+                                     __float_as_uint(__uint_as_float(rr[4 * u]) * p.scale),
+                                     __float_as_uint(__uint_as_float(rr[4 * u + 1]) * p.scale),
+                                     __float_as_uint(__uint_as_float(rr[4 * u + 2]) * p.scale),
+                                     __float_as_uint(__uint_as_float(rr[4 * u + 3]) * p.scale));
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(smem_u32(&ctl->stage_full));
+                if (t == 0) {
+                    // one thread adds the staged tile into the fp32 dQ buffer (rows past Tq
+                    // fall outside the tensor map and are dropped)
+                    if (!(ok = mbar_wait_bounded(smem_u32(&ctl->stage_full), rounds & 1u, abort_flag, p.err,
+                                                 p.timeout_ns)))
+                        break;
+                    const int plane = b * p.Hq + a;
+                    tma_reduce_add_3d(&tm_dq, sStage, h * 64, i * kBwdRows, plane);
+                    tma_reduce_add_3d(&tm_dq, sStage + kChunkBytes, h * 64 + 32, i * kBwdRows, plane);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(smem_u32(&ctl->stage_free));
                 }
             }
         }
+        if (t == 0) bulk_wait_all();  // every reduction into dQ has completed
         if (ok && mbar_wait_bounded(smem_u32(&ctl->dkdv_full), 0, abort_flag, p.err, p.timeout_ns)) {
             tc_fence_after_sync();
             const int key = j * kBwdKeys + t;

@@ -52,6 +52,22 @@ gqa_status make_map(CUtensorMap* map, const void* base, int B, int H, int T, int
     return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_UNSUPPORTED;
 }
 
+// The fp32 dQ buffer [BH, Tq, D] as a 3-D map (D, Tq, BH) with [128 rows][32 columns]
+// boxes in the 128-byte swizzle, for bulk reductions from shared memory. Rows past Tq of a
+// (b, head) plane fall outside the map and are never written.
+gqa_status make_dq_map(CUtensorMap* map, void* base, int BH, int Tq, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GQA_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Tq, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Tq * D * 4};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_UNSUPPORTED;
+}
+
 // Strides of a dimension of extent 1 are never used; give TMA a harmless legal value.
 long long effective_stride(long long s, int extent, long long fallback) {
     return extent == 1 ? fallback : s;
@@ -424,6 +440,7 @@ gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void*
     a.dq = dq; a.dk = dk; a.dv = dv;
     char* ws = static_cast<char*>(workspace);
     a.dq_acc = reinterpret_cast<float*>(ws);
+    if ((st = make_dq_map(&a.tm_dq, a.dq_acc, B * Hq, Tq, D)) != GQA_OK) return st;
     a.lse2 = reinterpret_cast<float*>(ws + dq_bytes);
     a.dvec = reinterpret_cast<float*>(ws + dq_bytes + vec_bytes);
     return gqa::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;

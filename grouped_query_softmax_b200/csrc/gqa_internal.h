@@ -70,7 +70,7 @@ struct DecLaunch {
 // Backward (gqa_attn_bwd). The workspace holds the fp32 dQ buffer, then LSE * log2(e)
 // and <dO, O> per query row padded to whole 128-row tiles.
 struct BwdLaunch {
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq;  // tm_dq: the fp32 dQ buffer, for bulk reductions
     int B, Hq, Hkv, Tq, Tk, D;
     float scale;
     const void* o;

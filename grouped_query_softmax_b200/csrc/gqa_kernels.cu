@@ -213,7 +213,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
         a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys), (unsigned)(a.B * a.Hkv));
-    gqa_bwd_sm100_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+    gqa_bwd_sm100_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long n8 = (long long)a.B * a.Hq * a.Tq * a.D / 8;
     gqa_bwd_dq_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.dq),
