@@ -418,10 +418,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after_sync();
 #pragma unroll 1
             for (int h = 0; h < D / 64 && ok; ++h, ++rounds) {
-                // the previous round's bulk reduction has finished reading the staging tile
-                if (rounds > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->stage_free), (rounds - 1) & 1u, abort_flag,
-                                                           p.err, p.timeout_ns)))
-                    break;
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tDP + lane_sel + h * 64, r0);
                 tmem_ld32(tDP + lane_sel + h * 64 + 32, r1);
@@ -433,6 +429,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tc_fence_before_sync();
                     mbar_arrive(smem_u32(&ctl->dq_empty));
                 }
+                // the previous round's bulk reduction has finished reading the staging tile
+                if (rounds > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->stage_free), (rounds - 1) & 1u, abort_flag,
+                                                           p.err, p.timeout_ns)))
+                    break;
                 // row t of two [128][32] fp32 boxes, 16-byte units in the 128-byte swizzle
 #pragma unroll
                 for (int bx = 0; bx < 2; ++bx) {
