@@ -50,7 +50,7 @@ struct BwdParams {
     int tq_pad;     // n_qt * 128: row stride of lse2 and dvec
     float scale;
     float scale_log2;     // scale * log2(e)
-    const float* lse2;    // [B, Hq, tq_pad]: the forward's LSE * log2(e); +inf past Tq
+    const float* lse2;    // [B, Hq, tq_pad]: -(the forward's LSE) * log2(e); -inf past Tq
     const float* dvec;    // [B, Hq, tq_pad]: <dO_i, O_i>; 0 past Tq
     float* dq_acc;        // [B, Hq, Tq, D] fp32, zeroed by the prep kernel
     __nv_bfloat16* dk;    // [B, Hkv, Tk, D]
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t sStage = sbase + L::kStageOff;
     const uint32_t sLse = sbase + L::kLseOff;
     const uint32_t sDvec = sbase + L::kDvecOff;
-    const float* lse_s = reinterpret_cast<const float*>(smem + L::kLseOff);
+    const float* nlse_s = reinterpret_cast<const float*>(smem + L::kLseOff);  // -LSE_i log2(e)
     const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvecOff);
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtlOff);
     volatile uint32_t* abort_flag = &ctl->abort;
@@ -341,28 +341,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->lse_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             tc_fence_after_sync();
-            float pr[128];
+            // P^T row in fp32 pairs (kept for dS); the next 32-column chunk of S^T is loaded
+            // while this one is exponentiated
+            uint64_t pr[64];
+            uint32_t sb[2][32];
+            const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+            tmem_ld32(tS + lane_sel, sb[0]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32];
-                tmem_ld32(tS + lane_sel + c * 32, sr);
                 tc_wait_ld();
-                reg_fence32(sr);
+                reg_fence32(sb[c & 1]);
+                if (c + 1 < 4) tmem_ld32(tS + lane_sel + (c + 1) * 32, sb[(c + 1) & 1]);
+                const uint32_t* sr = sb[c & 1];
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + e);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float4 l4 = *reinterpret_cast<const float4*>(nlse_s + c * 32 + e);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 4; u += 2) {
                         const int col = c * 32 + e + u;
-                        float x = ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lv[u]));
-                        if (diag && col < lim) x = 0.f;
-                        pr[col] = x;
+                        const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[e + u]), __uint_as_float(sr[e + u + 1])),
+                                                  sl2, u ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y));
+                        float x0, x1;
+                        f2_unpack(x, x0, x1);
+                        x0 = ex2_approx(x0);
+                        x1 = ex2_approx(x1);
+                        if (diag && col < lim) x0 = 0.f;
+                        if (diag && col + 1 < lim) x1 = 0.f;
+                        pr[col / 2] = f2_pack(x0, x1);
+                        pk[(e + u) / 2] = pack_bf16x2(x0, x1);
                     }
                 }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
                 tmem_st16(tS + lane_sel + c * 16, pk);
             }
             tc_wait_st();
@@ -375,22 +384,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                                   p.timeout_ns)))
                 break;
             tc_fence_after_sync();
+            tmem_ld32(tDP + lane_sel, sb[0]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t dr[32];
-                tmem_ld32(tDP + lane_sel + c * 32, dr);
                 tc_wait_ld();
-                reg_fence32(dr);
+                reg_fence32(sb[c & 1]);
+                if (c + 1 < 4) tmem_ld32(tDP + lane_sel + (c + 1) * 32, sb[(c + 1) & 1]);
+                const uint32_t* dr = sb[c & 1];
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + e);
-                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float ds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) ds[u] = pr[c * 32 + e + u] * (__uint_as_float(dr[e + u]) - dv4[u]);
-                    pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
-                    pk[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                    const uint64_t ds0 = f2_mul(pr[(c * 32 + e) / 2],
+                                                f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                                       f2_pack(d4.x, d4.y)));
+                    const uint64_t ds1 = f2_mul(pr[(c * 32 + e) / 2 + 1],
+                                                f2_sub(f2_pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])),
+                                                       f2_pack(d4.z, d4.w)));
+                    float a0, a1, a2, a3;
+                    f2_unpack(ds0, a0, a1);
+                    f2_unpack(ds1, a2, a3);
+                    pk[e / 2] = pack_bf16x2(a0, a1);
+                    pk[e / 2 + 1] = pack_bf16x2(a2, a3);
                 }
                 // row t, query columns c*32 .. c*32+31: four 16-byte units of chunk c/2
                 const uint32_t rowb = sDS + (uint32_t)((c >> 1) * kChunkBytes + t * 128);
@@ -502,8 +517,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
 }
 
-// D_i = <dO_i, O_i> and LSE_i * log2(e) per query row (padded to whole 128-row tiles with
-// 0 and +inf), and the fp32 dQ buffer zeroed. One warp per row.
+// D_i = <dO_i, O_i> and -LSE_i * log2(e) per query row (padded to whole 128-row tiles with
+// 0 and -inf), and the fp32 dQ buffer zeroed. One warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) gqa_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                            const __nv_bfloat16* __restrict__ dout,
@@ -517,7 +532,7 @@ __global__ void __launch_bounds__(256) gqa_bwd_prep_kernel(const __nv_bfloat16* 
     const int r = (int)(gw - bh * tq_pad);
     if (r >= Tq) {
         if (lane == 0) {
-            lse2[gw] = INFINITY;
+            lse2[gw] = -INFINITY;  // P = 2^(s - inf) = 0 for rows past Tq
             dvec[gw] = 0.f;
         }
         return;
@@ -533,7 +548,7 @@ __global__ void __launch_bounds__(256) gqa_bwd_prep_kernel(const __nv_bfloat16* 
     for (int e = 0; e < E; ++e) dq_acc[base + e] = 0.f;
     if (lane == 0) {
         dvec[gw] = acc;
-        lse2[gw] = lse[bh * Tq + r] * 1.4426950408889634f;
+        lse2[gw] = -lse[bh * Tq + r] * 1.4426950408889634f;
     }
 }
 
