@@ -425,14 +425,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int t = (warp - 8) * 32 + lane;
         const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
-        uint32_t rounds = 0;  // staging rounds so far (64 dQ columns each)
+        uint32_t rounds = 0;   // staging rounds so far (64 dQ columns each)
+        bool pending = false;  // thread 0: a bulk reduction whose shared-memory read is not yet released
+        // thread 0 waits until its last reduction has read the staging tile and frees the tile;
+        // it does so only right before the tile is needed again, so the TMEM columns of dQ
+        // are handed back to the MMA without waiting for the reduction
+        auto release = [&]() {
+            if (t == 0 && pending) {
+                bulk_wait_read_all();
+                mbar_arrive(smem_u32(&ctl->stage_free));
+                pending = false;
+            }
+        };
         for (int w = 0; w < items && ok; ++w) {
             const int i = i0 + w / p.G;
             const int a = g * p.G + (w - (w / p.G) * p.G);
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->dq_full), w & 1u, abort_flag, p.err, p.timeout_ns))) break;
             tc_fence_after_sync();
 #pragma unroll 1
-            for (int h = 0; h < D / 64 && ok; ++h, ++rounds) {
+            for (int h = 0; h < D / 64 && ok; ++h) {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tDP + lane_sel + h * 64, r0);
                 tmem_ld32(tDP + lane_sel + h * 64 + 32, r1);
@@ -445,6 +456,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mbar_arrive(smem_u32(&ctl->dq_empty));
                 }
                 // the previous round's bulk reduction has finished reading the staging tile
+                release();
                 if (rounds > 0 && !(ok = mbar_wait_bounded(smem_u32(&ctl->stage_free), (rounds - 1) & 1u, abort_flag,
                                                            p.err, p.timeout_ns)))
                     break;
@@ -473,9 +485,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tma_reduce_add_3d(&tm_dq, sStage, h * 64, i * kBwdRows, plane);
                     tma_reduce_add_3d(&tm_dq, sStage + kChunkBytes, h * 64 + 32, i * kBwdRows, plane);
                     bulk_commit_group();
-                    bulk_wait_read_all();
-                    mbar_arrive(smem_u32(&ctl->stage_free));
+                    pending = true;
                 }
+                ++rounds;
             }
         }
         if (t == 0) bulk_wait_all();  // every reduction into dQ has completed
