@@ -35,9 +35,16 @@ import numpy as np  # noqa: E402
 import gqa_inputs as gi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["grouped_query_softmax_b200/csrc/fwd_sm100.cuh", "grouped_query_softmax_b200/csrc/bwd_sm100.cuh",
-                  "grouped_query_softmax_b200/csrc/decode_sm100.cuh",
-                  "grouped_query_softmax_b200/csrc/sm100_ptx.cuh"]
+_CSRC = "grouped_query_softmax_b200/csrc/"
+# The sources each kernel is compiled from: a traffic figure stays valid while these hash
+# to the value recorded with it.
+KERNEL_SOURCES = {
+    "gqa_fwd_sm100_kernel": [_CSRC + "fwd_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gqa_decode_sm100_kernel": [_CSRC + "decode_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gqa_bwd_sm100_kernel": [_CSRC + "bwd_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
+}
+KERNEL_SOURCES["gqa_fwd_sm100_kernel_varlen"] = KERNEL_SOURCES["gqa_fwd_sm100_kernel"]
+KERNEL_SOURCES["gqa_decode_sm100_kernel_varlen"] = KERNEL_SOURCES["gqa_decode_sm100_kernel"]
 
 
 # ---------------------------------------------------------------- work counts
@@ -75,9 +82,9 @@ def is_decode(w) -> bool:
     return w.Tq <= 16 and w.Tk >= 1024
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, p), "rb").read())
     return h.hexdigest()[:16]
 
@@ -98,7 +105,7 @@ def load_traffic(kernel: str, workload: str):
         return None
     d = json.load(open(path))
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+    if not e or e.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 

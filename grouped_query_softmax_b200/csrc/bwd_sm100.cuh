@@ -530,35 +530,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // D_i = <dO_i, O_i> and -LSE_i * log2(e) per query row (padded to whole 128-row tiles with
-// 0 and -inf), and the fp32 dQ buffer zeroed. One warp per row.
+// 0 and -inf), and the fp32 dQ buffer zeroed. D / 8 lanes per row, 16-byte accesses.
 template <int D>
 __global__ void __launch_bounds__(256) gqa_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                            const __nv_bfloat16* __restrict__ dout,
                                                            const float* __restrict__ lse, float* __restrict__ lse2,
                                                            float* __restrict__ dvec, float* __restrict__ dq_acc,
                                                            int BH, int Tq, int tq_pad) {
-    const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (gw >= (long long)BH * tq_pad) return;
+    constexpr int kLanes = D / 8;            // lanes per row (16 or 8), 8 elements each
+    constexpr int kRows = 256 / kLanes;      // rows per block
+    const int sub = threadIdx.x % kLanes;
+    const long long gw = (long long)blockIdx.x * kRows + threadIdx.x / kLanes;
+    if (gw >= (long long)BH * tq_pad) return;  // whole row groups leave together
     const long long bh = gw / tq_pad;
     const int r = (int)(gw - bh * tq_pad);
     if (r >= Tq) {
-        if (lane == 0) {
+        if (sub == 0) {
             lse2[gw] = -INFINITY;  // P = 2^(s - inf) = 0 for rows past Tq
             dvec[gw] = 0.f;
         }
         return;
     }
-    constexpr int E = D / 32;  // elements per lane
-    const size_t base = ((size_t)bh * Tq + r) * D + lane * E;
+    const size_t base = ((size_t)bh * Tq + r) * D + sub * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(o + base);
+    const uint4 dv = *reinterpret_cast<const uint4*>(dout + base);
+    const uint32_t* ow = reinterpret_cast<const uint32_t*>(&ov);
+    const uint32_t* dw = reinterpret_cast<const uint32_t*>(&dv);
     float acc = 0.f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(o[base + e]), __bfloat162float(dout[base + e]), acc);
+    for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(dw[e] << 16), acc);
+        acc = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(dw[e] & 0xFFFF0000u), acc);
+    }
+    // only this row's lanes take part (other rows of the warp may have left)
+    const unsigned group = (kLanes == 32 ? 0xffffffffu : ((1u << kLanes) - 1u)) << ((threadIdx.x & 31) & ~(kLanes - 1));
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-#pragma unroll
-    for (int e = 0; e < E; ++e) dq_acc[base + e] = 0.f;
-    if (lane == 0) {
+    for (int s = kLanes / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(group, acc, s);
+    float4* z = reinterpret_cast<float4*>(dq_acc + base);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sub == 0) {
         dvec[gw] = acc;
         lse2[gw] = -lse[bh * Tq + r] * 1.4426950408889634f;
     }

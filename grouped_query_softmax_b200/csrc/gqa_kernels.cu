@@ -208,7 +208,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split needs it
     const long long rows = (long long)a.B * a.Hq * p.tq_pad;
-    gqa_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+    constexpr int kPrepRows = 256 / (D / 8);
+    gqa_bwd_prep_kernel<D><<<(unsigned)((rows + kPrepRows - 1) / kPrepRows), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.lse2, a.dvec,
         a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
