@@ -92,7 +92,7 @@ _lib.gqa_attn_decode_varlen.argtypes = ([_vp] * 6 + [_i32] * 9 + [_lay] * 2 + [_
 _lib.gqa_attn_bwd_workspace_bytes.restype = _sz
 _lib.gqa_attn_bwd_workspace_bytes.argtypes = [_i32] * 6
 _lib.gqa_attn_bwd.restype = _i32
-_lib.gqa_attn_bwd.argtypes = [_vp] * 9 + [_i32] * 6 + [_ll] * 4 + [_f32, _vp, _sz, _vp]
+_lib.gqa_attn_bwd.argtypes = [_vp] * 9 + [_i32] * 6 + [_ll] * 4 + [_f32, _i32, _vp, _sz, _vp]
 _lib.gqa_status_string.restype = ctypes.c_char_p
 _lib.gqa_status_string.argtypes = [_i32]
 _lib.gqa_get_device_error.restype = _i32
@@ -215,10 +215,10 @@ def gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Tq, Tk, D) -> int:
 
 
 def gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
-                 softmax_scale=0.0, workspace=None, workspace_bytes=0, stream=None) -> int:
+                 softmax_scale=0.0, window=0, workspace=None, workspace_bytes=0, stream=None) -> int:
     """C ``gqa_attn_bwd``: dq, dk, dv of the causal GQA forward for the output gradient dout."""
     return _lib.gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
-                             float(softmax_scale), workspace, workspace_bytes, stream)
+                             float(softmax_scale), int(window), workspace, workspace_bytes, stream)
 
 
 def gqa_status_string(status: int) -> str:
@@ -465,8 +465,8 @@ def attn_decode_varlen(q, k_cache, v_cache, seqlens_k, *, block_table=None, max_
     return out
 
 
-def attn_bwd(q, k, v, o, dout, lse, *, Tk=None, scale=None, dq=None, dk=None, dv=None, workspace=None,
-             stream=None):
+def attn_bwd(q, k, v, o, dout, lse, *, Tk=None, scale=None, window=0, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
     """Gradients (dq, dk, dv) of ``attn_fwd(q, k, v)`` for the output gradient ``dout``.
 
     o and lse are the forward's output and its log-sum-exp (``attn_fwd(..., return_lse=True)``);
@@ -494,7 +494,8 @@ def attn_bwd(q, k, v, o, dout, lse, *, Tk=None, scale=None, dq=None, dk=None, dv
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     st = gqa_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
-                      float(scale or 0.0), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+                      float(scale or 0.0), int(window), workspace.data_ptr(), workspace.numel(),
+                      _stream_handle(stream))
     if st != GQA_OK:
         raise GqaError(st, "gqa_attn_bwd")
     return dq, dk, dv

@@ -14,7 +14,7 @@
 // dV accumulate in TMEM for the whole group without atomics. Per step, with K_j and V_j
 // resident in shared memory:
 //   S^T  = K_j Q_i^T      (tcgen05, TMEM; lanes = keys)
-//   P^T  = 2^(S^T scale log2e - LSE_i log2e), causal mask on the diagonal tiles (bf16, in place)
+//   P^T  = 2^(S^T scale log2e - LSE_i log2e), causal (and window) mask on the edge tiles (bf16, in place)
 //   dP^T = V_j dO_i^T     (TMEM)
 //   dV  += P^T dO_i       (A from TMEM)
 //   dS^T = P^T (dP^T - D_i)  -> shared memory, bf16, [keys][rows]
@@ -57,6 +57,7 @@ struct BwdParams {
     __nv_bfloat16* dv;    // [B, Hkv, Tk, D]
     uint32_t* err;
     unsigned long long timeout_ns;
+    int window;     // > 0: each query sees only its `window` most recent positions
 };
 
 template <int D>
@@ -97,7 +98,16 @@ __device__ __forceinline__ int bwd_first_tile(int j, int Tq, int Tk) {
     return r > 0 ? r / kBwdRows : 0;
 }
 
-template <int D>
+// One past the last query tile with a row that sees key block j: with a window w, row r
+// (position Tk - Tq + r) sees keys down to position - w + 1 only.
+__device__ __forceinline__ int bwd_end_tile(int j, int Tq, int Tk, int n_qt, int window) {
+    if (window <= 0) return n_qt;
+    const int r_last = j * kBwdKeys + kBwdKeys - 1 + window - 1 - (Tk - Tq);  // last row seeing the block
+    if (r_last < 0) return 0;
+    return min(n_qt, r_last / kBwdRows + 1);
+}
+
+template <int D, bool kWindow>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     gqa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -135,7 +145,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int g = bg - b * p.Hkv;
     const int off = p.Tk - p.Tq;
     const int i0 = bwd_first_tile(j, p.Tq, p.Tk);
-    const int items = p.G * (p.n_qt - i0);  // (query tile, head) steps, tile-major
+    const int i1 = kWindow ? bwd_end_tile(j, p.Tq, p.Tk, p.n_qt, p.window) : p.n_qt;
+    // (query tile, head) steps, tile-major; 0 when no query sees the block (inside a window)
+    const int items = i1 > i0 ? p.G * (i1 - i0) : 0;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl->kv_full), 1);
@@ -335,9 +347,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int i = i0 + w / p.G;
             const int a = g * p.G + (w - (w / p.G) * p.G);
             (void)a;
-            // column c (query row i*128 + c) sees this key iff c >= lim
+            // column c (query row i*128 + c) sees this key iff lim <= c < lim + window
             const int lim = kabs - (off + i * kBwdRows);
-            const bool diag = j * kBwdKeys + kBwdKeys - 1 > off + i * kBwdRows;
+            const int lim_hi = kWindow ? lim + p.window : 0;
+            const bool diag = j * kBwdKeys + kBwdKeys - 1 > off + i * kBwdRows ||
+                              (kWindow && off + i * kBwdRows + kBwdRows - p.window > j * kBwdKeys);
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->lse_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             if (!(ok = mbar_wait_bounded(smem_u32(&ctl->s_full), ph, abort_flag, p.err, p.timeout_ns))) break;
             tc_fence_after_sync();
@@ -366,8 +380,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         f2_unpack(x, x0, x1);
                         x0 = ex2_approx(x0);
                         x1 = ex2_approx(x1);
-                        if (diag && col < lim) x0 = 0.f;
-                        if (diag && col + 1 < lim) x1 = 0.f;
+                        if (diag && (col < lim || (kWindow && col >= lim_hi))) x0 = 0.f;
+                        if (diag && (col + 1 < lim || (kWindow && col + 1 >= lim_hi))) x1 = 0.f;
                         pr[col / 2] = f2_pack(x0, x1);
                         pk[(e + u) / 2] = pack_bf16x2(x0, x1);
                     }
@@ -491,7 +505,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
         if (t == 0) bulk_wait_all();  // every reduction into dQ has completed
-        if (ok && mbar_wait_bounded(smem_u32(&ctl->dkdv_full), 0, abort_flag, p.err, p.timeout_ns)) {
+        if (kWindow && ok && items == 0) {
+            // no query sees this key block (it lies before every row's window): zero gradients
+            const int key = j * kBwdKeys + t;
+            if (key < p.Tk) {
+                const size_t orow = ((size_t)b * p.Hkv + g) * p.Tk + key;
+                uint4* k4 = reinterpret_cast<uint4*>(p.dk + orow * D);
+                uint4* v4 = reinterpret_cast<uint4*>(p.dv + orow * D);
+#pragma unroll
+                for (int e = 0; e < D / 8; ++e) k4[e] = v4[e] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else if (ok && mbar_wait_bounded(smem_u32(&ctl->dkdv_full), 0, abort_flag, p.err, p.timeout_ns)) {
             tc_fence_after_sync();
             const int key = j * kBwdKeys + t;
             const size_t orow = ((size_t)b * p.Hkv + g) * p.Tk + key;

@@ -414,9 +414,11 @@ size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int 
 gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                         const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Tq, int Tk,
                         int D, long long k_sb, long long k_sh, long long v_sb, long long v_sh,
-                        float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+                        float softmax_scale, int window, void* workspace, size_t workspace_bytes,
+                        void* stream) {
     gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
     if (st != GQA_OK) return st;
+    if (window < 0) return GQA_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
         !aligned16(dk) || !aligned16(dv) || !aligned16(lse))
         return GQA_ERR_INVALID_ARGUMENT;
@@ -435,6 +437,7 @@ gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void*
     if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
     if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.window = window >= Tk ? 0 : window;  // a window covering every key is plain causal
     a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
     a.o = o; a.dout = dout; a.lse = lse;
     a.dq = dq; a.dk = dk; a.dv = dv;

@@ -72,6 +72,7 @@ struct DecLaunch {
 struct BwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq;  // tm_dq: the fp32 dQ buffer, for bulk reductions
     int B, Hq, Hkv, Tq, Tk, D;
+    int window;
     float scale;
     const void* o;
     const void* dout;

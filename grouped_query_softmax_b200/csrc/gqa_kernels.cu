@@ -179,7 +179,7 @@ cudaError_t launch_decode(const DecLaunch& a, cudaStream_t stream) {
     return a.D == 128 ? launch_decode_d<128, false>(a, stream) : launch_decode_d<64, false>(a, stream);
 }
 
-template <int D>
+template <int D, bool kWindow>
 static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
     BwdParams p{};
     p.B = a.B;
@@ -190,6 +190,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
     p.G = a.Hq / a.Hkv;
     p.n_qt = (a.Tq + kBwdRows - 1) / kBwdRows;
     p.tq_pad = p.n_qt * kBwdRows;
+    p.window = a.window;
     p.scale = a.scale;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.lse2 = a.lse2;
@@ -201,10 +202,10 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
     p.timeout_ns = kWaitTimeoutNs;
     if (!p.err) return cudaErrorUnknown;
     const int smem = BwdSmem<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(gqa_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(gqa_bwd_sm100_kernel<D, kWindow>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaFuncAttributes fa{};
-    e = cudaFuncGetAttributes(&fa, gqa_bwd_sm100_kernel<D>);
+    e = cudaFuncGetAttributes(&fa, gqa_bwd_sm100_kernel<D, kWindow>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split needs it
     const long long rows = (long long)a.B * a.Hq * p.tq_pad;
@@ -214,7 +215,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
         a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys), (unsigned)(a.B * a.Hkv));
-    gqa_bwd_sm100_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
+    gqa_bwd_sm100_kernel<D, kWindow><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long n8 = (long long)a.B * a.Hq * a.Tq * a.D / 8;
     gqa_bwd_dq_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(a.dq_acc, static_cast<__nv_bfloat16*>(a.dq),
@@ -223,7 +224,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd(const BwdLaunch& a, cudaStream_t stream) {
-    return a.D == 128 ? launch_bwd_d<128>(a, stream) : launch_bwd_d<64>(a, stream);
+    if (a.window > 0) return a.D == 128 ? launch_bwd_d<128, true>(a, stream) : launch_bwd_d<64, true>(a, stream);
+    return a.D == 128 ? launch_bwd_d<128, false>(a, stream) : launch_bwd_d<64, false>(a, stream);
 }
 
 // One CTA, one thread: wait on an mbarrier that never completes, bounded by

@@ -289,15 +289,18 @@ GQA_API gqa_status gqa_attn_decode_varlen(const void* q, const void* k_cache, co
  *   workspace   device, >= gqa_attn_bwd_workspace_bytes(...) bytes, 256-byte aligned
  *               (an fp32 copy of dQ plus two fp32 values per query row); contents on
  *               entry ignored; not shared by calls that can overlap on the GPU.
- * Causal only (no window). dQ is accumulated with fp32 atomic additions, so its last
- * bits can differ from run to run; dK and dV are deterministic.
+ *   window      0 = causal; > 0 = the sliding window of gqa_attn_fwd_ex (the forward
+ *               that produced o and lse must have used the same window).
+ * dQ is accumulated with fp32 bulk additions in arrival order, so its last bits can differ
+ * from run to run; dK and dV are deterministic. Keys that no query sees (before every
+ * row's window) get zero gradients.
  */
 GQA_API size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D);
 GQA_API gqa_status gqa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
                                 int B, int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb,
                                 long long k_sh, long long v_sb, long long v_sh, float softmax_scale,
-                                void* workspace, size_t workspace_bytes, void* stream);
+                                int window, void* workspace, size_t workspace_bytes, void* stream);
 
 /* A static, human-readable name for a status code. */
 GQA_API const char* gqa_status_string(gqa_status s);

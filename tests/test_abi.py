@@ -184,7 +184,7 @@ def test_varlen_decode_split_planning(gqa):
 
 def bwd(gqa, **kw):
     a = dict(q=P, k=P, v=P, o=P, dout=P, lse=P, dq=P, dk=P, dv=P, B=1, Hq=4, Hkv=2, Tq=8, Tk=8, D=64,
-             k_sb=2 * 8 * 64, k_sh=8 * 64, v_sb=2 * 8 * 64, v_sh=8 * 64, softmax_scale=0.0,
+             k_sb=2 * 8 * 64, k_sh=8 * 64, v_sb=2 * 8 * 64, v_sh=8 * 64, softmax_scale=0.0, window=0,
              workspace=P, workspace_bytes=1 << 20, stream=None)
     a.update(kw)
     return gqa.gqa_attn_bwd(**a)
@@ -193,7 +193,7 @@ def bwd(gqa, **kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(Hq=3), 1), (dict(Tq=9), 1), (dict(dk=None), 1), (dict(lse=P + 4), 1), (dict(D=96), 2),
     (dict(k_sh=8 * 64 + 4), 1), (dict(workspace=None), 3), (dict(workspace_bytes=16), 3),
-    (dict(workspace=P + 64), 3),
+    (dict(workspace=P + 64), 3), (dict(window=-1), 1),
 ])
 def test_bwd_rejects_bad_arguments(gqa, kw, status):
     assert bwd(gqa, **kw) == status

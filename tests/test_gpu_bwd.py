@@ -93,3 +93,53 @@ def test_bwd_full_size_gqa_prefill(gqa):
     assert_grad_parity(from_dev(dq[:1]), rq, "dQ gqa_prefill b0")
     assert_grad_parity(from_dev(dk[:1]), rk, "dK gqa_prefill b0")
     assert_grad_parity(from_dev(dv[:1]), rv, "dV gqa_prefill b0")
+
+
+WINDOW_CASES = [
+    # B, Hq, Hkv, Tq, Tk, D, window
+    (1, 4, 2, 700, 700, 128, 200),     # window inside tiles
+    (2, 6, 2, 300, 1500, 128, 128),    # suffix far after the prefix: early key blocks unseen (zero grads)
+    (1, 8, 1, 513, 513, 64, 8),        # a window much shorter than a tile
+]
+# Windows of 1 or 2 keys are left to the test below: there dS = P (dP - D) is a difference of
+# near-equal terms and D = <dO, O> from the bf16 output carries a rounding error of the same
+# size (inherent to forming D from O), so an error bar relative to dQ's own size is too tight.
+
+
+@pytest.mark.parametrize("case", WINDOW_CASES, ids=[str(c) for c in WINDOW_CASES])
+def test_bwd_window_matches_oracle(gqa, case):
+    B, Hq, Hkv, Tq, Tk, D, win = case
+    w = gi.Workload("bwd window", B, Hq, Hkv, Tq, Tk, D, seed=117)
+    q, k, v = w.make()
+    do = w.make_dout()
+    qd, kd, vd, dod = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    o, lse = gqa.attn_fwd(qd, kd, vd, window=win, return_lse=True)
+    dq, dk, dv = gqa.attn_bwd(qd, kd, vd, o, dod, lse, window=win)
+    torch_mod().cuda.synchronize()
+    assert gqa.gqa_get_device_error() == gqa.GQA_OK
+    rq, rk, rv = oracle.attention_bwd(q, k, v, do, window=win)
+    assert_grad_parity(from_dev(dq), rq, f"dQ {case}")
+    assert_grad_parity(from_dev(dk), rk, f"dK {case}")
+    assert_grad_parity(from_dev(dv), rv, f"dV {case}")
+    if case[4] - case[3] > 2 * case[6] + 128:
+        # keys that no query sees have exactly zero gradients
+        unseen = Tk - Tq - win
+        assert (from_dev(dk)[:, :, :unseen] == 0).all() and (from_dev(dv)[:, :, :unseen] == 0).all()
+
+
+def test_bwd_window_of_one_has_no_score_gradient(gqa):
+    """With w = 1 every row sees only itself: P = 1, so dS = dP - <dO, o> = 0 exactly and dQ,
+    dK vanish; dV_j = dO of the query at position j. A bar relative to a zero reference is
+    empty, so dQ and dK are checked against the size of dV instead."""
+    w = gi.Workload("bwd window 1", 1, 8, 1, 513, 513, 64, seed=119)
+    q, k, v = w.make()
+    do = w.make_dout()
+    qd, kd, vd, dod = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    o, lse = gqa.attn_fwd(qd, kd, vd, window=1, return_lse=True)
+    dq, dk, dv = gqa.attn_bwd(qd, kd, vd, o, dod, lse, window=1)
+    torch_mod().cuda.synchronize()
+    assert gqa.gqa_get_device_error() == gqa.GQA_OK
+    _, _, rv = oracle.attention_bwd(q, k, v, do, window=1)
+    assert_grad_parity(from_dev(dv), rv, "dV window 1")
+    scale = float(np.abs(rv).max())
+    assert np.abs(from_dev(dq)).max() <= MAX_REL * scale and np.abs(from_dev(dk)).max() <= MAX_REL * scale
