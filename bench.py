@@ -329,6 +329,45 @@ def varlen_flops(w) -> float:
     return 4.0 * w.D * w.Hq * sum(visible_pairs(int(a), int(b), w.window) for a, b in zip(lq, lk) if a)
 
 
+def measure_paged_prefill(w, page, steps, warmup, world, dev):
+    """The chunked-prefill workload with each sequence's keys in a paged pool (pages of
+    `page` keys in a seeded random order, [pages, page, Hkv, D])."""
+    import torch
+    import grouped_query_softmax_b200 as gqa
+    q, k, v, cu_q, cu_k = w.make()
+    lq, lk = w.lengths()
+    n_pages = (lk + page - 1) // page
+    order = gi.permutation(w.seed, gi.STREAM_PAGES, int(n_pages.sum()))
+    pool_k = np.zeros((order.size, page, w.Hkv, w.D), dtype=np.uint16)
+    pool_v = np.zeros_like(pool_k)
+    table = np.full((w.S, int(n_pages.max())), -1, dtype=np.int32)
+    at = 0
+    for s in range(w.S):
+        for i in range(int(n_pages[s])):
+            pg = order[at]
+            at += 1
+            table[s, i] = pg
+            r0, r1 = int(cu_k[s]) + i * page, int(cu_k[s]) + min((i + 1) * page, int(lk[s]))
+            pool_k[pg, :r1 - r0] = k[r0:r1]
+            pool_v[pg, :r1 - r0] = v[r0:r1]
+    qd, kd, vd = to_device(q, dev), to_device(pool_k, dev), to_device(pool_v, dev)
+    cq = torch.tensor(cu_q, device=dev)
+    ld = torch.tensor(lk.astype(np.int32), device=dev)
+    td = torch.tensor(table, device=dev)
+    od = torch.empty_like(qd)
+    max_q = int(lq.max())
+    ws = torch.empty(gqa.gqa_attn_fwd_varlen_workspace_bytes(w.S, w.Hq, w.Hkv, max_q), dtype=torch.uint8, device=dev)
+    fn = lambda: gqa.attn_fwd_varlen(qd, kd, vd, cu_seqlens_q=cq, seqlens_k=ld, block_table=td, max_seqlen_q=max_q,
+                                     window=w.window, out=od, workspace=ws)
+    ms, _, _ = timed(fn, steps, warmup, world, dev)
+    st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
+    if st != gqa.GQA_OK:
+        raise RuntimeError(f"device error after paged prefill timing: {gqa.gqa_status_string(st)}")
+    del qd, kd, vd, od, ws
+    torch.cuda.empty_cache()
+    return {"ms_total": ms, "launches": 2 * steps}
+
+
 def paged_kv_bytes(w) -> int:
     """K + V bytes of every cached key, read once per KV head."""
     return 2 * int(w.lengths().sum()) * w.Hkv * w.D * 2
@@ -759,6 +798,18 @@ def main(argv=None):
                              "traffic": load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
                 "gpu_launches": rv["launches"]}
+        # the chunked-prefill workload again, its keys read from a paged pool
+        wv = gi.VARLEN_WORKLOADS["chunked_prefill"]
+        rpp = measure_paged_prefill(wv, 64, nsv, max(3, args.warmup), world, dev)
+        mspp = rpp["ms_total"] / nsv
+        achpp = varlen_flops(wv) / (mspp * 1e-3) / 1e12
+        line["paged_chunked_prefill"] = {
+            "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achpp, "unit": "TFLOP/s",
+            "ms_per_step": mspp, "config": varlen_config(wv) | {"keys": "paged, 64 per page, seeded random page order"},
+            "roofline": {"bound": "tensor", "achieved": achpp, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achpp / peaks["bf16_tflops"], "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+            "gpu_launches": rpp["launches"]}
         # backward (training) on the headline workload
         nsb = max(10, args.steps // 4)
         rb = measure_bwd(w, nsb, max(3, args.warmup), world, dev)

@@ -23,7 +23,7 @@ __all__ = [
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
     "GqaLayout", "gqa_attn_fwd_varlen", "gqa_attn_fwd_varlen_workspace_bytes", "gqa_attn_decode_varlen",
     "gqa_attn_decode_varlen_workspace_bytes", "gqa_attn_decode_varlen_num_splits",
-    "gqa_attn_bwd", "gqa_attn_bwd_workspace_bytes", "attn_bwd",
+    "gqa_attn_bwd", "gqa_attn_bwd_workspace_bytes", "attn_bwd", "gqa_attn_fwd_varlen_paged",
     "attn_fwd_varlen", "attn_decode_varlen",
     "GQA_OK", "GQA_ERR_INVALID_ARGUMENT", "GQA_ERR_UNSUPPORTED", "GQA_ERR_WORKSPACE",
     "GQA_ERR_CUDA", "GQA_ERR_TIMEOUT",
@@ -83,6 +83,8 @@ _lib.gqa_attn_fwd_varlen_workspace_bytes.restype = _sz
 _lib.gqa_attn_fwd_varlen_workspace_bytes.argtypes = [_i32] * 4
 _lib.gqa_attn_fwd_varlen.restype = _i32
 _lib.gqa_attn_fwd_varlen.argtypes = ([_vp] * 9 + [_i32] * 7 + [_lay] * 4 + [_f32, _i32, _vp, _sz, _vp])
+_lib.gqa_attn_fwd_varlen_paged.restype = _i32
+_lib.gqa_attn_fwd_varlen_paged.argtypes = ([_vp] * 9 + [_i32] * 9 + [_lay] * 4 + [_f32, _i32, _vp, _sz, _vp])
 _lib.gqa_attn_decode_varlen_workspace_bytes.restype = _sz
 _lib.gqa_attn_decode_varlen_workspace_bytes.argtypes = [_i32] * 8
 _lib.gqa_attn_decode_varlen_num_splits.restype = _i32
@@ -188,6 +190,19 @@ def gqa_attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, seqlens_q, 
                                     S, Hq, Hkv, D, rows_q, rows_k, max_seqlen_q, ctypes.byref(lq),
                                     ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
                                     float(softmax_scale), int(window), workspace, workspace_bytes, stream)
+
+
+def gqa_attn_fwd_varlen_paged(q, k_pool, v_pool, o, lse, cu_seqlens_q, seqlens_q, seqlens_k, block_table,
+                              page_size, num_pages, max_pages, S, Hq, Hkv, D, rows_q, max_seqlen_q, q_layout,
+                              k_layout, v_layout, o_layout, softmax_scale=0.0, window=0, workspace=None,
+                              workspace_bytes=0, stream=None) -> int:
+    """C ``gqa_attn_fwd_varlen_paged``: variable-length forward over a paged key/value cache."""
+    lq, lk, lv, lo = (_layout(x) for x in (q_layout, k_layout, v_layout, o_layout))
+    return _lib.gqa_attn_fwd_varlen_paged(q, k_pool, v_pool, o, lse, cu_seqlens_q, seqlens_q, seqlens_k,
+                                          block_table, page_size, num_pages, max_pages, S, Hq, Hkv, D, rows_q,
+                                          max_seqlen_q, ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv),
+                                          ctypes.byref(lo), float(softmax_scale), int(window), workspace,
+                                          workspace_bytes, stream)
 
 
 def gqa_attn_decode_varlen_workspace_bytes(B, Hq, Hkv, Tq, max_seqlen_k, D, window=0, num_splits=0) -> int:
@@ -350,7 +365,7 @@ def _int32_cuda(t, name):
 
 def attn_fwd_varlen(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, seqlens_q=None, seqlens_k=None,
                     max_seqlen_q=None, scale=None, window=0, return_lse=False, out=None, workspace=None,
-                    stream=None):
+                    block_table=None, pool_layout="NHD", stream=None):
     """S independent causal GQA problems of different lengths in one call.
 
     Each side is packed, a 3-D [rows, H, D] tensor (any row/head strides, so token-major
@@ -359,7 +374,14 @@ def attn_fwd_varlen(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, seqlens_q=
     lengths ``seqlens_*`` [S]. Sequence s's L_q query rows sit at positions L_k - L_q ..
     L_k - 1 of its own keys. Returns o shaped like q (rows of no sequence untouched)
     and, with ``return_lse``, the fp32 LSE [Hq, rows_q] (packed) or [S, Hq, rows_q].
+
+    With ``block_table`` (int32 [S, max_pages]) the keys are paged: k and v are pools
+    [pages, page, Hkv, D] ("NHD") or [pages, Hkv, page, D] ("HND") and ``seqlens_k`` gives
+    each sequence's key count.
     """
+    if block_table is not None:
+        return _attn_fwd_varlen_paged(q, k, v, cu_seqlens_q, seqlens_q, seqlens_k, block_table, max_seqlen_q,
+                                      scale, window, return_lse, out, workspace, pool_layout, stream)
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_bf16_cuda(t, n)
@@ -499,3 +521,54 @@ def attn_bwd(q, k, v, o, dout, lse, *, Tk=None, scale=None, window=0, dq=None, d
     if st != GQA_OK:
         raise GqaError(st, "gqa_attn_bwd")
     return dq, dk, dv
+
+
+def _attn_fwd_varlen_paged(q, k_pool, v_pool, cu_seqlens_q, seqlens_q, seqlens_k, block_table, max_seqlen_q,
+                           scale, window, return_lse, out, workspace, pool_layout, stream):
+    torch = _torch()
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _check_bf16_cuda(t, n)
+    cu_q = _int32_cuda(cu_seqlens_q, "cu_seqlens_q")
+    len_q, len_k = _int32_cuda(seqlens_q, "seqlens_q"), _int32_cuda(seqlens_k, "seqlens_k")
+    table = _int32_cuda(block_table, "block_table")
+    if len_k is None:
+        raise ValueError("a paged cache needs seqlens_k")
+    packed_q, rows_q, Hq, lay_q = _side_layout(q, "q")
+    if packed_q != (cu_q is not None):
+        raise ValueError("packed (3-D) queries need cu_seqlens_q; padded (4-D) queries must not have it")
+    if k_pool.shape != v_pool.shape or k_pool.dim() != 4 or k_pool.stride(3) != 1:
+        raise ValueError("k_pool and v_pool must be 4-D with a contiguous D axis and equal shapes")
+    if pool_layout == "NHD":
+        num_pages, page, Hkv, D = k_pool.shape
+        lay = lambda t: (t.stride(0), t.stride(2), t.stride(1))
+    elif pool_layout == "HND":
+        num_pages, Hkv, page, D = k_pool.shape
+        lay = lambda t: (t.stride(0), t.stride(1), t.stride(2))
+    else:
+        raise ValueError("pool_layout must be 'NHD' or 'HND'")
+    S = cu_q.numel() - 1 if packed_q else q.shape[0]
+    if table.dim() != 2 or table.shape[0] != S or len_k.numel() != S:
+        raise ValueError("block_table must be [S, max_pages] and seqlens_k [S]")
+    if max_seqlen_q is None:
+        if packed_q:
+            max_seqlen_q = int((cu_q[1:] - cu_q[:-1]).max().item())
+        else:
+            max_seqlen_q = int(len_q.max().item()) if len_q is not None else rows_q
+    max_seqlen_q = max(1, int(max_seqlen_q))
+    if out is None:
+        out = torch.empty_like(q)
+    _, _, _, lay_o = _side_layout(out, "out")
+    lse = None
+    if return_lse:
+        lse = torch.empty(((Hq, rows_q) if packed_q else (S, Hq, rows_q)), dtype=torch.float32, device=q.device)
+    need = gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = gqa_attn_fwd_varlen_paged(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), out.data_ptr(), _ptr(lse),
+                                   _ptr(cu_q), _ptr(len_q), len_k.data_ptr(), table.data_ptr(), page, num_pages,
+                                   table.shape[1], S, Hq, Hkv, D, rows_q, max_seqlen_q, lay_q, lay(k_pool),
+                                   lay(v_pool), lay_o, float(scale or 0.0), int(window), workspace.data_ptr(),
+                                   workspace.numel(), _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_fwd_varlen_paged")
+    return (out, lse) if return_lse else out

@@ -79,6 +79,10 @@ struct FwdVarlenParams {
     const int* unit_list;   // present units, longest first (written by the plan kernel)
     const int* unit_count;  // their number
     long long o_sb, o_sh, o_st;  // element strides of o (batch, head, row); d is contiguous
+    // paged keys (table non-null): key t of sequence s is row t % page_size of pool page
+    // table[s * max_pages + t / page_size]; the k/v tensor maps cover the pool
+    const int* table;
+    int max_pages, page_size, box_rows, num_pages;
 };
 
 // Where one sequence's rows are: batch index, first row and length of each side.
@@ -351,9 +355,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         const uint32_t fbar = smem_u32(ragged ? &ctl->land[stage] : &ctl->full[stage]);
                         mbar_arrive_expect_tx(fbar, kTileBytes);
                         const CUtensorMap* map = t ? &tm_v : &tm_k;
-                        for (int c = 0; c < L::kChunks; ++c)
-                            tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
-                                        geo.r_k + j * kFwdKeys, g, geo.b_k);
+                        if (kVarlen && vp.table != nullptr) {
+                            // one box per page (or per 128 keys of a large page); keys past the
+                            // sequence read an out-of-range page, i.e. zeros
+                            const int n_box = kFwdKeys / vp.box_rows;
+                            for (int bi = 0; bi < n_box; ++bi) {
+                                const int key0 = j * kFwdKeys + bi * vp.box_rows;
+                                const int page = key0 < geo.len_k
+                                                     ? __ldg(vp.table + (size_t)geo.b_k * vp.max_pages + key0 / vp.page_size)
+                                                     : vp.num_pages;
+                                const uint32_t dst = sRing + stage * kTileBytes + bi * vp.box_rows * 128;
+                                for (int c = 0; c < L::kChunks; ++c)
+                                    tma_load_4d(dst + c * kChunkBytes, map, fbar, c * 64, key0 % vp.page_size, g, page);
+                            }
+                        } else {
+                            for (int c = 0; c < L::kChunks; ++c)
+                                tma_load_4d(sRing + stage * kTileBytes + c * kChunkBytes, map, fbar, c * 64,
+                                            geo.r_k + j * kFwdKeys, g, geo.b_k);
+                        }
                         ++issued[stage];
                         if constexpr (kVarlen) {
                             last_land[stage] = ragged;

@@ -287,13 +287,18 @@ size_t gqa_attn_fwd_varlen_workspace_bytes(int S, int Hq, int Hkv, int max_seqle
     return gqa::fwd_varlen_workspace_bytes(n);
 }
 
-gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
-                               const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqlens_q,
-                               const int* seqlens_k, int S, int Hq, int Hkv, int D, int rows_q,
-                               int rows_k, int max_seqlen_q, const gqa_layout* q_layout,
-                               const gqa_layout* k_layout, const gqa_layout* v_layout,
-                               const gqa_layout* o_layout, float softmax_scale, int window,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Shared by the contiguous and the paged variable-length forward. table non-null: the keys
+// are paged (rows_k = the key capacity, max_pages * page_size; the k/v layouts and maps cover
+// the pool of num_pages pages).
+gqa_status fwd_varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                           const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqlens_q,
+                           const int* seqlens_k, const int* table, int page_size, int num_pages, int max_pages,
+                           int S, int Hq, int Hkv, int D, int rows_q, int rows_k, int max_seqlen_q,
+                           const gqa_layout* q_layout, const gqa_layout* k_layout, const gqa_layout* v_layout,
+                           const gqa_layout* o_layout, float softmax_scale, int window, void* workspace,
+                           size_t workspace_bytes, void* stream) {
     if (S <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || rows_q <= 0 || rows_k <= 0 || max_seqlen_q <= 0)
         return GQA_ERR_INVALID_ARGUMENT;
     if (Hq % Hkv != 0 || window < 0) return GQA_ERR_INVALID_ARGUMENT;
@@ -303,21 +308,23 @@ gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
     if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
     const int bq = cu_seqlens_q ? 1 : S;  // batch extent of each side
-    const int bk = cu_seqlens_k ? 1 : S;
+    const int bk = table ? num_pages : (cu_seqlens_k ? 1 : S);
+    const int kv_rows = table ? page_size : rows_k;  // rows of one k/v batch plane (a page)
     gqa::FwdVarlenLaunch a{};
     long long ls[3][3];  // (sb, sh, st) of q, k, v
     gqa_status e;
     if ((e = check_layout(q_layout, bq, Hq, rows_q, D, ls[0][0], ls[0][1], ls[0][2])) != GQA_OK) return e;
-    if ((e = check_layout(k_layout, bk, Hkv, rows_k, D, ls[1][0], ls[1][1], ls[1][2])) != GQA_OK) return e;
-    if ((e = check_layout(v_layout, bk, Hkv, rows_k, D, ls[2][0], ls[2][1], ls[2][2])) != GQA_OK) return e;
+    if ((e = check_layout(k_layout, bk, Hkv, kv_rows, D, ls[1][0], ls[1][1], ls[1][2])) != GQA_OK) return e;
+    if ((e = check_layout(v_layout, bk, Hkv, kv_rows, D, ls[2][0], ls[2][1], ls[2][2])) != GQA_OK) return e;
     if ((e = check_layout(o_layout, bq, Hq, rows_q, D, a.o_sb, a.o_sh, a.o_st)) != GQA_OK) return e;
     const size_t need = gqa_attn_fwd_varlen_workspace_bytes(S, Hq, Hkv, max_seqlen_q);
     if (need == 0) return GQA_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return GQA_ERR_WORKSPACE;
     if ((e = make_map(&a.tm_q, q, bq, Hq, rows_q, D, ls[0][0], ls[0][1], ls[0][2])) != GQA_OK) return e;
-    if ((e = make_map(&a.tm_k, k, bk, Hkv, rows_k, D, ls[1][0], ls[1][1], ls[1][2])) != GQA_OK) return e;
-    if ((e = make_map(&a.tm_v, v, bk, Hkv, rows_k, D, ls[2][0], ls[2][1], ls[2][2])) != GQA_OK) return e;
+    const int box = table && page_size < gqa::kTileKeys ? page_size : gqa::kTileKeys;
+    if ((e = make_map(&a.tm_k, k, bk, Hkv, kv_rows, D, ls[1][0], ls[1][1], ls[1][2], box)) != GQA_OK) return e;
+    if ((e = make_map(&a.tm_v, v, bk, Hkv, kv_rows, D, ls[2][0], ls[2][1], ls[2][2], box)) != GQA_OK) return e;
     a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D;
     a.rows_q = rows_q; a.rows_k = rows_k; a.max_q = max_seqlen_q;
     a.window = window;
@@ -327,7 +334,43 @@ gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void
     a.o = o;
     a.lse = lse;
     a.ws = static_cast<int*>(workspace);
+    a.table = table;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    a.max_pages = max_pages;
     return gqa::launch_fwd_varlen(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+
+gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, const int* seqlens_q,
+                               const int* seqlens_k, int S, int Hq, int Hkv, int D, int rows_q,
+                               int rows_k, int max_seqlen_q, const gqa_layout* q_layout,
+                               const gqa_layout* k_layout, const gqa_layout* v_layout,
+                               const gqa_layout* o_layout, float softmax_scale, int window,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    return fwd_varlen_impl(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, seqlens_q, seqlens_k, nullptr, 0, 0, 0, S,
+                           Hq, Hkv, D, rows_q, rows_k, max_seqlen_q, q_layout, k_layout, v_layout, o_layout,
+                           softmax_scale, window, workspace, workspace_bytes, stream);
+}
+
+gqa_status gqa_attn_fwd_varlen_paged(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
+                                     const int* cu_seqlens_q, const int* seqlens_q, const int* seqlens_k,
+                                     const int* block_table, int page_size, int num_pages, int max_pages, int S,
+                                     int Hq, int Hkv, int D, int rows_q, int max_seqlen_q,
+                                     const gqa_layout* q_layout, const gqa_layout* k_layout,
+                                     const gqa_layout* v_layout, const gqa_layout* o_layout, float softmax_scale,
+                                     int window, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!seqlens_k || !block_table) return GQA_ERR_INVALID_ARGUMENT;
+    const bool page_ok = page_size >= 16 && page_size % 16 == 0 &&
+                         (page_size % gqa::kTileKeys == 0 || gqa::kTileKeys % page_size == 0);
+    if (!page_ok || num_pages <= 0 || max_pages <= 0) return GQA_ERR_INVALID_ARGUMENT;
+    if ((long long)max_pages * page_size > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
+    return fwd_varlen_impl(q, k_pool, v_pool, o, lse, cu_seqlens_q, nullptr, seqlens_q, seqlens_k, block_table,
+                           page_size, num_pages, max_pages, S, Hq, Hkv, D, rows_q, max_pages * page_size,
+                           max_seqlen_q, q_layout, k_layout, v_layout, o_layout, softmax_scale, window, workspace,
+                           workspace_bytes, stream);
 }
 
 int gqa_attn_decode_varlen_num_splits(int B, int Hq, int Hkv, int Tq, int max_seqlen_k, int D, int window,

@@ -33,6 +33,9 @@ struct FwdVarlenLaunch {
     long long o_sb, o_sh, o_st;  // elements
     float* lse;
     int* ws;  // plan workspace (fwd_varlen_workspace_bytes)
+    // paged keys (gqa_attn_fwd_varlen_paged); table null = contiguous keys
+    const int* table;
+    int max_pages, page_size, num_pages;
 };
 
 // Candidate units of a variable-length forward: S x row levels x head slots. A unit

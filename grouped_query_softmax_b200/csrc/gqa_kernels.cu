@@ -103,6 +103,11 @@ static cudaError_t launch_fwd_varlen_d(const FwdVarlenLaunch& a, cudaStream_t st
     vp.o_sb = a.o_sb;
     vp.o_sh = a.o_sh;
     vp.o_st = a.o_st;
+    vp.table = a.table;
+    vp.max_pages = a.max_pages;
+    vp.page_size = a.page_size;
+    vp.box_rows = a.page_size > 0 && a.page_size < kFwdKeys ? a.page_size : kFwdKeys;
+    vp.num_pages = a.num_pages;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;

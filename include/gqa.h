@@ -230,6 +230,30 @@ GQA_API gqa_status gqa_attn_fwd_varlen(const void* q, const void* k, const void*
                                        size_t workspace_bytes, void* stream);
 
 /*
+ * gqa_attn_fwd_varlen over a paged key/value cache (chunked prefill reading the same pages
+ * the decode steps use). Queries are packed (cu_seqlens_q) or padded (seqlens_q), as for
+ * gqa_attn_fwd_varlen. Sequence s holds seqlens_k[s] keys (int32 [S] on the device,
+ * required); key t of sequence s is row t % page_size of pool page
+ * block_table[s * max_pages + t / page_size] (int32 [S, max_pages] on the device).
+ *   k_pool, v_pool  bf16 pools of num_pages pages, element (page, h, r, d) at
+ *                   page*sb + h*sh + r*st + d (k_layout / v_layout).
+ *   page_size       16, 32, 64 or a multiple of 128.
+ * Every seqlens_k[s] must lie within max_pages * page_size (checked on the device, reported
+ * like the other bounds). Table entries past a sequence's last page are never read; a page
+ * number outside [0, num_pages) reads zeros; key rows past a sequence's length (the rest of
+ * its last page) may hold any bits. Other arguments as for gqa_attn_fwd_varlen; the
+ * workspace is sized by gqa_attn_fwd_varlen_workspace_bytes.
+ */
+GQA_API gqa_status gqa_attn_fwd_varlen_paged(const void* q, const void* k_pool, const void* v_pool, void* o,
+                                             float* lse, const int* cu_seqlens_q, const int* seqlens_q,
+                                             const int* seqlens_k, const int* block_table, int page_size,
+                                             int num_pages, int max_pages, int S, int Hq, int Hkv, int D,
+                                             int rows_q, int max_seqlen_q, const gqa_layout* q_layout,
+                                             const gqa_layout* k_layout, const gqa_layout* v_layout,
+                                             const gqa_layout* o_layout, float softmax_scale, int window,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode over a cache whose sequences have different lengths, contiguous or paged.
  * Sequence b holds L(b) = seqlens_k[b] keys; its T_q new queries are the last T_q of
  * them (positions L(b) - T_q .. L(b) - 1), as for gqa_attn_decode_ex. Each sequence's

@@ -203,3 +203,23 @@ def test_bwd_workspace_size(gqa):
     # fp32 dQ [B,Hq,Tq,D] + two fp32 values per row padded to 128-row tiles, each 256-aligned
     assert gqa.gqa_attn_bwd_workspace_bytes(1, 4, 2, 8, 8, 64) == 8192 + 2 * 2048
     assert gqa.gqa_attn_bwd_workspace_bytes(1, 4, 2, 9, 8, 64) == 0
+
+
+def paged_fwd(gqa, **kw):
+    lay_q = (0, 64, 4 * 64)
+    lay_kv = (64 * 2 * 64, 64, 2 * 64)   # pool [pages, 64, 2, 64] (NHD)
+    a = dict(q=P, k_pool=P, v_pool=P, o=P, lse=None, cu_seqlens_q=P, seqlens_q=None, seqlens_k=P,
+             block_table=P, page_size=64, num_pages=10, max_pages=4, S=2, Hq=4, Hkv=2, D=64, rows_q=64,
+             max_seqlen_q=40, q_layout=lay_q, k_layout=lay_kv, v_layout=lay_kv, o_layout=lay_q,
+             softmax_scale=0.0, window=0, workspace=P, workspace_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_fwd_varlen_paged(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(seqlens_k=None), 1), (dict(block_table=None), 1), (dict(page_size=48), 1), (dict(page_size=8), 1),
+    (dict(num_pages=0), 1), (dict(max_pages=0), 1), (dict(k_layout=(64 * 2 * 64, 64, 100)), 1),
+    (dict(workspace=None), 3), (dict(seqlens_q=P), 1),
+])
+def test_paged_fwd_rejects_bad_arguments(gqa, kw, status):
+    assert paged_fwd(gqa, **kw) == status

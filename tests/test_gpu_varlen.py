@@ -290,3 +290,34 @@ def test_full_size_paged_decode_workload(gqa):
         vc = ov.gather_pages(hnd_v, table[b:b + 1], lens[b:b + 1], w.page)
         ref = oracle.attention(np.ascontiguousarray(q[b:b + 1]), kc, vc)
         assert_parity(got[b:b + 1], ref, f"paged decode sequence {b}")
+
+
+PAGED_PREFILL = [
+    # chunk lengths, cached-prefix lengths, Hq, Hkv, D, page, pool layout, window
+    ([300, 1, 640], [700, 0, 1000], 8, 2, 128, 16, "NHD", 0),
+    ([129, 512], [127, 1500], 8, 1, 128, 64, "HND", 0),
+    ([700, 200, 33], [0, 900, 4000], 6, 2, 128, 256, "NHD", 300),
+    ([257, 100], [600, 77], 4, 4, 64, 128, "NHD", 0),
+]
+
+
+@pytest.mark.parametrize("case", PAGED_PREFILL, ids=[str(c) for c in PAGED_PREFILL])
+def test_chunked_prefill_over_a_paged_cache(gqa, case):
+    """New tokens packed, every sequence's keys (its cached prefix and the chunk itself)
+    in a shuffled page pool; rest-of-page rows and spare pages hold NaN."""
+    lq, pre, Hq, Hkv, D, page, layout, w = case
+    lq, lk = np.array(lq), np.array(pre) + np.array(lq)
+    S, T = len(lq), int(lk.max())
+    cu_q = gi.cu_from_lengths(lq)
+    q = gi.normal_bf16(89, gi.TENSOR_Q, (int(cu_q[-1]), Hq, D))
+    k = gi.normal_bf16(89, gi.TENSOR_K, (S, Hkv, T, D))
+    v = gi.normal_bf16(89, gi.TENSOR_V, (S, Hkv, T, D))
+    for s in range(S):
+        k[s, :, lk[s]:] = NAN_BITS
+        v[s, :, lk[s]:] = NAN_BITS
+    pk, pv, table = _paged_pool(k, v, lk, page, seed=91, layout=layout)
+    o = gqa.attn_fwd_varlen(to_dev(q), to_dev(pk), to_dev(pv), cu_seqlens_q=_i32(cu_q), seqlens_k=_i32(lk),
+                            block_table=_i32(table), pool_layout=layout, window=w)
+    _sync_ok(gqa)
+    ref = ov.attention_varlen(_head_major(q), k, v, S, cu_q=cu_q, len_k=lk, window=w)
+    _check_packed(from_dev(o), ref, cu_q, f"paged prefill {case}")
