@@ -496,8 +496,8 @@ gqa_status gqa_get_device_error(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
     uint32_t v = 0;
     if (gqa::read_and_clear_device_error(&v) != cudaSuccess) return GQA_ERR_CUDA;
-    if (v & 1u) return GQA_ERR_TIMEOUT;  // a bounded wait ran out
-    if (v & 2u) return GQA_ERR_INVALID_ARGUMENT;  // sequence bounds outside their tensors
+    if (v & gqa::kErrBitWaitTimeout) return GQA_ERR_TIMEOUT;
+    if (v & gqa::kErrBitBadSeqlens) return GQA_ERR_INVALID_ARGUMENT;
     return GQA_OK;
 }
 

@@ -105,6 +105,10 @@ cudaError_t launch_selftest_wait(unsigned long long timeout_ns, cudaStream_t str
 // Read and clear the device error word of the current device (after a stream sync).
 cudaError_t read_and_clear_device_error(uint32_t* value);
 
+// Bits of the device error word (set by the kernels, read by gqa_get_device_error).
+constexpr uint32_t kErrBitWaitTimeout = 1u;   // a bounded wait ran out
+constexpr uint32_t kErrBitBadSeqlens = 2u;    // sequence bounds outside their tensors
+
 // Bound on every device-side wait of the production kernels.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 

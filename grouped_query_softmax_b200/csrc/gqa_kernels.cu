@@ -12,7 +12,9 @@
 
 namespace gqa {
 
-// Bit flags (kDevErr*) set by bounded waits that ran out; see gqa_get_device_error().
+// Bit flags (kDevErr*) set by the kernels; see gqa_get_device_error().
+static_assert(kDevErrWaitTimeout == kErrBitWaitTimeout && kDevErrBadSeqlens == kErrBitBadSeqlens,
+              "device and host disagree on the error bits");
 __device__ uint32_t g_device_error = 0;
 
 static uint32_t* device_error_ptr() {

@@ -1,0 +1,60 @@
+"""bench.py's host-side arithmetic (CPU only): the work counts behind every roofline
+figure, checked against brute-force enumeration, and the peak and traffic bookkeeping."""
+import json
+import os
+
+import numpy as np
+
+import bench
+import gqa_inputs as gi
+
+
+def brute_pairs(Tq, Tk, window=0):
+    n = 0
+    for i in range(Tq):
+        pos = Tk - Tq + i
+        lo = max(0, pos - window + 1) if window > 0 else 0
+        n += pos - lo + 1
+    return n
+
+
+def test_visible_pairs_match_enumeration():
+    for Tq, Tk, w in [(1, 1, 0), (5, 5, 0), (3, 10, 0), (7, 7, 3), (4, 20, 6), (9, 9, 100), (1, 32768, 0)]:
+        assert bench.visible_pairs(Tq, Tk, w) == brute_pairs(Tq, Tk, w), (Tq, Tk, w)
+
+
+def test_flop_and_byte_counts():
+    w = gi.WORKLOADS["gqa_prefill"]
+    assert bench.algorithmic_flops(w) == 4.0 * 128 * 32 * 4 * (4096 * 4097 // 2)
+    assert abs(bench.bwd_flops(w) / bench.algorithmic_flops(w) - 2.5) < 1e-12
+    d = gi.WORKLOADS["gqa_decode"]
+    assert bench.kv_bytes(d) == 2 * 64 * 8 * 32768 * 128 * 2
+    vw = gi.VARLEN_WORKLOADS["chunked_prefill"]
+    lq, lk = vw.lengths()
+    want = 4.0 * vw.D * vw.Hq * sum(brute_pairs(int(a), int(b)) for a, b in zip(lq, lk))
+    assert bench.varlen_flops(vw) == want
+    pw = gi.VARLEN_WORKLOADS["paged_decode"]
+    assert bench.paged_kv_bytes(pw) == 2 * int(pw.lengths().sum()) * pw.Hkv * pw.D * 2
+
+
+def test_tensor_peak_follows_the_power_cap():
+    peaks = {"bf16_tflops": 1630.1, "bf16_tflops_sustained": 1374.1}
+    assert bench.tensor_peak(peaks, "measured", {"reasons": []})[0] == 1630.1
+    assert bench.tensor_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})[0] == 1374.1
+    assert "sustained" in bench.tensor_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})[1]
+    assert bench.tensor_peak({"bf16_tflops": 1590.0}, "fallback", {"reasons": ["sw_power_cap"]})[0] == 1590.0
+
+
+def test_traffic_figures_follow_their_kernel_sources():
+    path = os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")
+    table = json.load(open(path))
+    for kernel, entries in table.items():
+        if kernel.startswith("_"):
+            continue
+        assert kernel in bench.KERNEL_SOURCES
+        for workload, e in entries.items():
+            got = bench.load_traffic(kernel, workload)
+            fresh = e["kernel_source_hash"] == bench.kernel_source_hash(kernel)
+            assert (got == e["dram_bytes_per_launch"]) if fresh else got is None
+            assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
+    assert bench.load_traffic("gqa_fwd_sm100_kernel", "no such workload") is None
