@@ -100,6 +100,18 @@ def tensor_peak(peaks, peak_src, clocks):
     return burst, f"{peak_src} bf16_tflops (burst; kernel timed alone)"
 
 
+def tensor_roofline(achieved, peaks, peak_src, clocks, traffic, kernel):
+    """The roofline object of a tensor-bound row: the power-cap-aware peak and the fraction
+    of it, with the fractions of the burst and sustained figures for context."""
+    peak, src = tensor_peak(peaks, peak_src, clocks)
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic, "peak_source": src,
+            "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+            "frac_of_spec_2250": achieved / 2250.0, "kernel": kernel}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -602,12 +614,9 @@ def backward_main(args, rank, world, local, dev, peaks, peak_src, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(w, {"pass": "backward (dQ, dK, dV)", "l2": "inputs larger than L2 (no flush)",
                                           "parallelism": f"dp{world} (independent problems per rank)"}),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak(peaks, peak_src, clocks)[0],
-                         "unit": "TFLOP/s", "frac": achieved / tensor_peak(peaks, peak_src, clocks)[0],
-                         "frac_of_burst": achieved / peaks["bf16_tflops"],
-                         "traffic": load_traffic("gqa_bwd_sm100_kernel", w.name),
-                         "peak_source": tensor_peak(peaks, peak_src, clocks)[1],
-                         "kernel": "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"},
+            "roofline": tensor_roofline(achieved, peaks, peak_src, clocks,
+                                        load_traffic("gqa_bwd_sm100_kernel", w.name),
+                                        "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"),
             "gpu_launches": r["launches"], "clocks": clocks}
     if world > 1:
         import torch.distributed as dist
@@ -640,21 +649,25 @@ def varlen_main(args, rank, world, local, dev, peaks, peak_src):
         work, unit, scale = varlen_flops(w), "TFLOP/s", 1e12
         metric = "GQA varlen prefill TFLOP/s on 1 B200, % of roofline"
         config = varlen_config(w) | {"tokens_q": r["tokens_q"], "tokens_k": r["tokens_k"]}
-        peak, bound, src = None, "tensor", None  # chosen from the clocks below
+        peak, bound, src = None, "tensor", None  # tensor_roofline below chooses the peak
         kernel = "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen>"
     ms_step = r["ms_total"] / args.steps
     achieved = work / (ms_step * 1e-3) / scale
     clocks = sampler.summary(r["t0"], r["t1"])
     sampler.stop()
-    if peak is None:
-        peak, src = tensor_peak(peaks, peak_src, clocks)
+    if bound == "tensor":
+        roof = tensor_roofline(achieved, peaks, peak_src, clocks,
+                               load_traffic("gqa_fwd_sm100_kernel_varlen", w.name), kernel)
+    else:
+        roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": load_traffic("gqa_decode_sm100_kernel_varlen", w.name), "peak_source": src,
+                "kernel": kernel}
     line = {"metric": metric, "value": world * achieved, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config | {"l2": "inputs larger than L2 (no flush)",
                                 "parallelism": f"dp{world} (independent problems per rank)"},
-            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": None, "peak_source": src, "kernel": kernel},
+            "roofline": roof,
             "gpu_launches": r["launches"], "clocks": clocks}
     if args.e2e_steps:
         e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
@@ -716,10 +729,6 @@ def main(argv=None):
     e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
     clocks = sampler.summary(r["t0"], r["t1"])
 
-    # A run that held the GPU at its power cap is compared with the sustained (power-capped)
-    # GEMM figure; otherwise with the burst figure. The extension rows use the same choice.
-    burst = peaks["bf16_tflops"]
-    tpeak, tsrc = tensor_peak(peaks, peak_src, clocks)
     if is_decode(w):
         per_launch_bytes = kv_bytes(w) + qo_bytes(w)
         achieved = per_launch_bytes / (ms_step * 1e-3) / 1e9
@@ -730,14 +739,8 @@ def main(argv=None):
                 "kernel": "gqa_decode_sm100_kernel + gqa_decode_combine_kernel (one call per step)"}
     else:
         achieved = algorithmic_flops(w) / (ms_step * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
-                "frac": achieved / tpeak,
-                "traffic": load_traffic("gqa_fwd_sm100_kernel", w.name),
-                "peak_source": tsrc,
-                "frac_of_burst": achieved / burst,
-                "frac_of_sustained": achieved / sustained,
-                "frac_of_spec_2250": achieved / 2250.0,
-                "kernel": "gqa_fwd_sm100_kernel"}
+        roof = tensor_roofline(achieved, peaks, peak_src, clocks,
+                               load_traffic("gqa_fwd_sm100_kernel", w.name), "gqa_fwd_sm100_kernel")
 
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -776,8 +779,7 @@ def main(argv=None):
         line["swa_prefill"] = {
             "metric": "TFLOP/s (window-visible pairs)", "value": throughput(ws_, mss, world),
             "unit": "TFLOP/s", "ms_per_step": mss, "config": workload_config(ws_),
-            "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": ach / tpeak, "frac_of_burst": ach / burst, "traffic": None, "peak_source": tsrc},
+            "roofline": tensor_roofline(ach, peaks, peak_src, clocks, None, "gqa_fwd_sm100_kernel<window>"),
             "gpu_launches": rs["launches"]}
         wc = gi.WORKLOADS["chunk_decode"]
         nst = max(3, args.steps // 20)
@@ -803,10 +805,9 @@ def main(argv=None):
                 "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achv,
                 "unit": "TFLOP/s", "ms_per_step": msv,
                 "config": varlen_config(wv) | {"tokens_q": rv["tokens_q"], "tokens_k": rv["tokens_k"]},
-                "roofline": {"bound": "tensor", "achieved": achv, "peak": tpeak,
-                             "unit": "TFLOP/s", "frac": achv / tpeak, "frac_of_burst": achv / burst,
-                             "traffic": load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
-                             "peak_source": tsrc},
+                "roofline": tensor_roofline(achv, peaks, peak_src, clocks,
+                                            load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
+                                            "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen>"),
                 "gpu_launches": rv["launches"]}
         # the chunked-prefill workload again, its keys read from a paged pool
         wv = gi.VARLEN_WORKLOADS["chunked_prefill"]
@@ -816,9 +817,8 @@ def main(argv=None):
         line["paged_chunked_prefill"] = {
             "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achpp, "unit": "TFLOP/s",
             "ms_per_step": mspp, "config": varlen_config(wv) | {"keys": "paged, 64 per page, seeded random page order"},
-            "roofline": {"bound": "tensor", "achieved": achpp, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": achpp / tpeak, "frac_of_burst": achpp / burst, "traffic": None,
-                         "peak_source": tsrc},
+            "roofline": tensor_roofline(achpp, peaks, peak_src, clocks, None,
+                                        "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen, paged>"),
             "gpu_launches": rpp["launches"]}
         # backward (training) on the headline workload
         nsb = max(10, args.steps // 4)
@@ -828,11 +828,9 @@ def main(argv=None):
         line["backward"] = {
             "metric": "TFLOP/s (10 * D * Hq * B * causal-visible pairs: S, dP, dV, dK, dQ)", "value": world * achb,
             "unit": "TFLOP/s", "ms_per_step": msb, "config": workload_config(w),
-            "roofline": {"bound": "tensor", "achieved": achb, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": achb / tpeak, "frac_of_burst": achb / burst,
-                         "traffic": load_traffic("gqa_bwd_sm100_kernel", w.name),
-                         "peak_source": tsrc,
-                         "kernel": "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"},
+            "roofline": tensor_roofline(achb, peaks, peak_src, clocks,
+                                        load_traffic("gqa_bwd_sm100_kernel", w.name),
+                                        "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"),
             "gpu_launches": rb["launches"]}
         wp = gi.VARLEN_WORKLOADS["paged_decode"]
         nsp = max(3, args.steps // 20)

@@ -58,3 +58,41 @@ def test_traffic_figures_follow_their_kernel_sources():
             assert (got == e["dram_bytes_per_launch"]) if fresh else got is None
             assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
     assert bench.load_traffic("gqa_fwd_sm100_kernel", "no such workload") is None
+
+
+def test_tensor_roofline_fractions():
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.tensor_roofline(700.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 123, "k")
+    assert r["peak"] == 1400.0 and r["frac"] == 0.5 and r["frac_of_burst"] == 700.0 / 1600.0
+    assert r["traffic"] == 123 and r["kernel"] == "k" and r["bound"] == "tensor"
+    r = bench.tensor_roofline(800.0, peaks, "measured", {"reasons": []}, None, "k")
+    assert r["peak"] == 1600.0 and r["frac"] == 0.5 and r["frac_of_sustained"] == 800.0 / 1400.0
+
+
+def _undefined_globals(path):
+    """Names that a function of the module reads as globals but that neither the module
+    nor the builtins define (what a static checker reports as an undefined name)."""
+    import builtins
+    import symtable
+    src = open(path, encoding="utf-8").read()
+    top = symtable.symtable(src, path, "exec")
+    defined = {s.get_name() for s in top.get_symbols() if s.is_assigned() or s.is_imported()}
+    defined |= set(dir(builtins)) | {"__file__", "__name__"}
+    missing = []
+
+    def walk(tab):
+        for sym in tab.get_symbols():
+            if sym.is_referenced() and sym.is_global() and sym.get_name() not in defined:
+                missing.append((tab.get_name(), tab.get_lineno(), sym.get_name()))
+        for child in tab.get_children():
+            walk(child)
+    for child in top.get_children():
+        walk(child)
+    return missing
+
+
+def test_host_scripts_have_no_undefined_names():
+    import __graft_entry__
+    import grouped_query_softmax_b200 as pkg
+    for path in (bench.__file__, __graft_entry__.__file__, pkg.__file__):
+        assert _undefined_globals(path) == [], path
