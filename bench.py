@@ -41,7 +41,7 @@ _CSRC = "grouped_query_softmax_b200/csrc/"
 KERNEL_SOURCES = {
     "gqa_fwd_sm100_kernel": [_CSRC + "fwd_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
     "gqa_decode_sm100_kernel": [_CSRC + "decode_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
-    "gqa_bwd_sm100_kernel": [_CSRC + "bwd_sm100.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gqa_bwd_sm100_kernel": [_CSRC + "bwd_sm100.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "gqa_internal.h"],
 }
 KERNEL_SOURCES["gqa_fwd_sm100_kernel_varlen"] = KERNEL_SOURCES["gqa_fwd_sm100_kernel"]
 KERNEL_SOURCES["gqa_decode_sm100_kernel_varlen"] = KERNEL_SOURCES["gqa_decode_sm100_kernel"]

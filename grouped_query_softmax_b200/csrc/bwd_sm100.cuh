@@ -29,6 +29,7 @@
 // TMEM (512 columns at D = 128): S^T | dP^T, later dQ | dV | dK.
 #pragma once
 
+#include "gqa_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace gqa {
@@ -46,6 +47,8 @@ static_assert(128 * (kBwdCtlRegs + kBwdPRegs + kBwdDqRegs) <= kBwdThreads * kBwd
 
 struct BwdParams {
     int B, Hq, Hkv, Tq, Tk, G;
+    int n_kb;       // key blocks per (batch, KV head)
+    int chunk;      // launch order: (batch, KV head) pairs per chunk (bwd_block_coords)
     int n_qt;       // ceil(Tq / 128)
     int tq_pad;     // n_qt * 128: row stride of lse2 and dvec
     float scale;
@@ -137,10 +140,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Key blocks of one (b, g) are launched together: they all add into the same dQ rows,
-    // which then stay in L2 while they run. Within a (b, g), low j first (most work).
-    const int j = blockIdx.x;
-    const int bg = blockIdx.y;  // b * Hkv + g
+    // Launch order: chunks of (b, g) pairs whose dQ rows stay in L2 while their key blocks
+    // add into them; inside a chunk, low j first (most work).
+    int j, bg;  // key block, b * Hkv + g
+    bwd_block_coords((int)blockIdx.x, p.n_kb, p.B * p.Hkv, p.chunk, &bg, &j);
     const int b = bg / p.Hkv;
     const int g = bg - b * p.Hkv;
     const int off = p.Tk - p.Tq;

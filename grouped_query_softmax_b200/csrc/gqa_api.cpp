@@ -501,6 +501,15 @@ gqa_status gqa_get_device_error(void* stream) {
     return GQA_OK;
 }
 
+gqa_status gqa_testing_bwd_order(int n_kb, int n_bg, int G, int Tq, int D, int* out_chunk, int* out_bg, int* out_j) {
+    if (n_kb <= 0 || n_bg <= 0 || G <= 0 || Tq <= 0 || D <= 0 || !out_chunk || !out_bg || !out_j)
+        return GQA_ERR_INVALID_ARGUMENT;
+    const int chunk = gqa::bwd_chunk(n_bg, G, Tq, D);
+    *out_chunk = chunk;
+    for (int L = 0; L < n_kb * n_bg; ++L) gqa::bwd_block_coords(L, n_kb, n_bg, chunk, &out_bg[L], &out_j[L]);
+    return GQA_OK;
+}
+
 gqa_status gqa_selftest_bounded_wait(unsigned long long timeout_ns, void* stream) {
     if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return GQA_ERR_INVALID_ARGUMENT;
     return gqa::launch_selftest_wait(timeout_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess

@@ -88,6 +88,30 @@ struct BwdLaunch {
     float* dvec;
 };
 
+// Backward launch order. Key block j of a (batch, KV head) pair walks the query tiles from
+// about j on, so low j carries the most work. The pairs are taken in chunks of `chunk`;
+// inside a chunk every pair's block 0 is launched first, then every pair's block 1, and so
+// on (longest first, which keeps the last wave short). A chunk's fp32 dQ rows, which all its
+// key blocks add into, are the L2 working set: `chunk` is the largest divisor of the number
+// of pairs whose dQ rows fit in kBwdChunkDqBytes.
+constexpr double kBwdChunkDqBytes = 72.0 * 1024 * 1024;
+inline int bwd_chunk(int n_bg, int G, int Tq, int D) {
+    const double per_pair = (double)G * Tq * D * sizeof(float);
+    int best = 1;
+    for (int c = 2; c <= n_bg; ++c)
+        if (n_bg % c == 0 && c * per_pair <= kBwdChunkDqBytes) best = c;
+    return best;
+}
+// (pair, key block) of linear block index L, for n_kb key blocks per pair.
+__host__ __device__ inline void bwd_block_coords(int L, int n_kb, int n_bg, int chunk, int* bg, int* j) {
+    const int per_chunk = chunk * n_kb;
+    const int c = L / per_chunk;
+    const int r = L - c * per_chunk;
+    const int width = n_bg - c * chunk < chunk ? n_bg - c * chunk : chunk;
+    *j = r / width;
+    *bg = c * chunk + (r - *j * width);
+}
+
 inline size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 inline void bwd_workspace_layout(int B, int Hq, int Tq, int D, size_t* dq_bytes, size_t* vec_bytes) {
     const size_t tq_pad = (size_t)(Tq + 127) / 128 * 128;

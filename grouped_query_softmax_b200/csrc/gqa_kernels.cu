@@ -195,6 +195,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
     p.Tq = a.Tq;
     p.Tk = a.Tk;
     p.G = a.Hq / a.Hkv;
+    p.n_kb = (a.Tk + kBwdKeys - 1) / kBwdKeys;
+    p.chunk = bwd_chunk(a.B * a.Hkv, p.G, a.Tq, D);
     p.n_qt = (a.Tq + kBwdRows - 1) / kBwdRows;
     p.tq_pad = p.n_qt * kBwdRows;
     p.window = a.window;
@@ -221,7 +223,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch& a, cudaStream_t stream) {
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.lse2, a.dvec,
         a.dq_acc, a.B * a.Hq, a.Tq, p.tq_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const dim3 grid((unsigned)((a.Tk + kBwdKeys - 1) / kBwdKeys), (unsigned)(a.B * a.Hkv));
+    const dim3 grid((unsigned)(p.n_kb * a.B * a.Hkv));
     gqa_bwd_sm100_kernel<D, kWindow><<<grid, kBwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long n8 = (long long)a.B * a.Hq * a.Tq * a.D / 8;

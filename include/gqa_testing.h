@@ -24,6 +24,17 @@ extern "C" {
  */
 GQA_API gqa_status gqa_selftest_bounded_wait(unsigned long long timeout_ns, void* stream);
 
+/*
+ * The launch order of the backward kernel's CTAs, for host-side tests. For n_kb key blocks
+ * of 128 keys per (batch, KV head) pair, n_bg pairs, G query heads per KV head, T_q query
+ * rows and head dimension D, writes *out_chunk (pairs per launch chunk) and, for every
+ * linear CTA index L < n_kb * n_bg, out_bg[L] and out_j[L]: the pair and the key block that
+ * CTA processes. The arrays are caller-owned host memory of n_kb * n_bg ints each. Touches
+ * no GPU. Returns GQA_ERR_INVALID_ARGUMENT for a non-positive size or a null pointer.
+ */
+GQA_API gqa_status gqa_testing_bwd_order(int n_kb, int n_bg, int G, int Tq, int D, int* out_chunk, int* out_bg,
+                                         int* out_j);
+
 #ifdef __cplusplus
 }
 #endif
