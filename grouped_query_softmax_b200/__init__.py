@@ -54,6 +54,11 @@ _lib.gqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _
 _lib.gqa_attn_fwd_ex.restype = _i32
 _lib.gqa_attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                  _ll, _ll, _ll, _ll, _f32, _i32, _vp]
+_lib.gqa_attn_fwd_host_workspace_bytes.restype = _sz
+_lib.gqa_attn_fwd_host_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
+_lib.gqa_attn_fwd_host.restype = _i32
+_lib.gqa_attn_fwd_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
+                                   _vp, _sz, _vp]
 _lib.gqa_attn_decode_workspace_bytes.restype = _sz
 _lib.gqa_attn_decode_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.gqa_attn_decode_num_splits.restype = _i32
@@ -126,6 +131,17 @@ def gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_
     """C ``gqa_attn_fwd_ex``: ``gqa_attn_fwd`` with a sliding window (0 = causal only)."""
     return _lib.gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
                                 float(softmax_scale), int(window), stream)
+
+
+def gqa_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Tq, Tk, D) -> int:
+    return int(_lib.gqa_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Tq, Tk, D))
+
+
+def gqa_attn_fwd_host(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, softmax_scale=0.0, window=0,
+                      workspace=None, workspace_bytes=0, stream=None) -> int:
+    """C ``gqa_attn_fwd_host``: q, k, v, o, lse are HOST addresses; workspace a device address."""
+    return _lib.gqa_attn_fwd_host(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, float(softmax_scale), int(window),
+                                  workspace, workspace_bytes, stream)
 
 
 def gqa_attn_decode_workspace_bytes(B, Hq, Hkv, Tk, D, num_splits=0) -> int:
@@ -304,6 +320,46 @@ def attn_fwd(q, k, v, *, Tk=None, scale=None, window=0, return_lse=False, out=No
                          _stream_handle(stream))
     if st != GQA_OK:
         raise GqaError(st, "gqa_attn_fwd_ex")
+    return (out, lse) if return_lse else out
+
+
+def attn_fwd_host(q, k, v, *, scale=None, window=0, return_lse=False, out=None, workspace=None, device=None,
+                  stream=None, synchronize=True):
+    """attn_fwd for operands in host memory: q [B,Hq,Tq,D] and k, v [B,Hkv,Tk,D], contiguous
+    bf16 CPU tensors (pinned, for the copies to overlap the kernels). The library streams
+    query-row chunks through a device workspace (gqa_attn_fwd_host) and writes o (and the
+    fp32 LSE) into CPU tensors. With ``synchronize=False`` the call returns once the work is
+    enqueued on ``stream``, and the outputs are valid once the stream reaches that point."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous bf16 CPU tensor")
+    B, Hq, Tq, D = q.shape
+    Hkv, Tk = k.shape[1], k.shape[2]
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("q, k, v shapes disagree")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 CPU tensor shaped like q")
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, pin_memory=q.is_pinned()) if return_lse else None
+    need = gqa_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Tq, Tk, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8,
+                                device=device if device is not None else torch.cuda.current_device())
+    st = gqa_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Tq, Tk, D,
+                           float(scale or 0.0), int(window), workspace.data_ptr(),
+                           workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != GQA_OK:
+        raise GqaError(st, "gqa_attn_fwd_host")
+    if synchronize:
+        if stream is None:
+            torch.cuda.current_stream().synchronize()
+        elif hasattr(stream, "synchronize"):
+            stream.synchronize()
+        else:
+            torch.cuda.synchronize()
     return (out, lse) if return_lse else out
 
 

@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgqa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["gqa_kernels.cu", "gqa_api.cpp", "gqa_decode_static.cu"]
+SOURCES = ["gqa_kernels.cu", "gqa_api.cpp", "gqa_decode_static.cu", "gqa_host.cpp"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -22,8 +22,9 @@
  * with V (the pages' reference rounds the fp32 probabilities to the input dtype
  * before "@ v"); O is rounded to bf16 round-to-nearest-even.
  *
- * Memory: every pointer is a DEVICE pointer owned by the caller. The library never
- * allocates device memory and keeps no per-call state; K and V are addressed per KV
+ * Memory: every pointer is a DEVICE pointer owned by the caller, except the operands of
+ * gqa_attn_fwd_host, which live in host memory. The library never allocates device
+ * memory and keeps no per-call state; K and V are addressed per KV
  * head and are never replicated per query head. All calls are asynchronous on
  * `stream` (a cudaStream_t; NULL = the legacy default stream) and return as soon as
  * the kernels are enqueued. Calls are thread-safe and re-entrant.
@@ -92,6 +93,43 @@ GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, 
                                    int B, int Hq, int Hkv, int Tq, int Tk, int D,
                                    long long k_sb, long long k_sh, long long v_sb, long long v_sh,
                                    float softmax_scale, int window, void* stream);
+
+/*
+ * gqa_attn_fwd_ex for operands in HOST memory, for callers whose tensors are not yet on the
+ * device. The pages define the operation only; moving operands is a library convenience.
+ *
+ * The query rows are cut into chunks of whole 128-row tiles, at most 8. Chunk c (rows
+ * [r0, r1)) is computed as the suffix call over keys [0, T_k - T_q + r1), the keys its rows
+ * see, so each query sits at the same position and gets the same result as in the one-shot
+ * call, bit for bit. Each key crosses to the device once, just before the first chunk that
+ * needs it. Copies in, the kernel and copies out run on three streams, so chunk c + 1's
+ * inputs and chunk c - 1's output move while chunk c is computed.
+ *
+ *   q, o     bf16 [B, Hq, Tq, D], contiguous host memory. Pinned memory (cudaHostAlloc or
+ *            cudaHostRegister) lets the copies overlap the kernels. With pageable memory the
+ *            results are the same, but the copies serialise.
+ *   k, v     bf16 [B, Hkv, Tk, D], contiguous host memory.
+ *   lse      NULL, or fp32 [B, Hq, Tq] host memory (as gqa_attn_fwd).
+ *   window   as gqa_attn_fwd_ex.
+ *   workspace  device memory of at least gqa_attn_fwd_host_workspace_bytes(...) bytes,
+ *            256-byte aligned. It holds K, V and two query/output slots. Its contents on
+ *            entry are ignored. It must not be used by other work that can overlap the call.
+ *   stream   the call is ordered on this stream. It starts after the work already enqueued
+ *            there. Work enqueued after it starts once every row of o (and lse) is in host
+ *            memory. The call returns without waiting, and the host buffers must stay
+ *            valid and unchanged until the stream gets there.
+ *
+ * Errors:
+ *   - Argument errors are reported as for gqa_attn_fwd_ex, before anything is enqueued.
+ *   - A missing, misaligned or short workspace returns GQA_ERR_WORKSPACE.
+ *   - GQA_ERR_CUDA means that a stream, event, copy or launch call failed. Part of the
+ *     work may then already be enqueued: synchronise the device before reusing o or the
+ *     workspace.
+ */
+GQA_API size_t gqa_attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D);
+GQA_API gqa_status gqa_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int Tq, int Tk, int D, float softmax_scale,
+                                     int window, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Decode (T_q = 1): the query of each (b, a) sits at position T_k - 1 and sees all

@@ -223,3 +223,38 @@ def paged_fwd(gqa, **kw):
 ])
 def test_paged_fwd_rejects_bad_arguments(gqa, kw, status):
     assert paged_fwd(gqa, **kw) == status
+
+
+H = 1 << 22  # a fake host address; these calls fail before touching memory or the GPU
+
+
+def fwd_host(gqa, **kw):
+    a = dict(q=H, k=H, v=H, o=H, lse=None, B=1, Hq=4, Hkv=2, Tq=300, Tk=300, D=64, softmax_scale=0.0, window=0,
+             workspace=P, workspace_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return gqa.gqa_attn_fwd_host(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(v=None), 1), (dict(o=None), 1),
+    (dict(Hq=3), 1), (dict(Tq=301), 1), (dict(window=-1), 1), (dict(softmax_scale=float("nan")), 1),
+    (dict(lse=H + 2), 1), (dict(D=96), 2),
+    (dict(workspace=None), 3), (dict(workspace=P + 128), 3), (dict(workspace_bytes=1024), 3),
+])
+def test_fwd_host_rejects_bad_arguments(gqa, kw, status):
+    assert fwd_host(gqa, **kw) == status
+
+
+def test_fwd_host_workspace_size(gqa):
+    # K and V whole, plus two slots of query rows, outputs and LSE; chunks of whole 128-row
+    # tiles, at most 8 of them and at least 256 rows each
+    def rnd(x):
+        return (x + 255) // 256 * 256
+    for B, Hq, Hkv, Tq, Tk, D in [(4, 32, 8, 4096, 4096, 128), (1, 4, 2, 300, 700, 64), (2, 8, 8, 100, 100, 128),
+                                  (1, 32, 1, 32768, 32768, 128)]:
+        rows = max(256, -(-(-(-Tq // 8)) // 128) * 128)
+        rows = min(rows, Tq)
+        want = 2 * rnd(B * Hkv * Tk * D * 2) + 2 * (2 * rnd(B * Hq * rows * D * 2) + rnd(B * Hq * rows * 4))
+        assert gqa.gqa_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Tq, Tk, D) == want
+    assert gqa.gqa_attn_fwd_host_workspace_bytes(1, 3, 2, 8, 8, 64) == 0
+    assert gqa.gqa_attn_fwd_host_workspace_bytes(1, 4, 2, 8, 8, 80) == 0
