@@ -315,20 +315,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 // the next step's S^T now: it runs while this step's dS is formed (the tensor
                 // pipe executes in order, so dV has read P^T before S^T overwrites it)
                 if (w + 1 < items && !(ok = issue_s(w + 1))) break;
-                // dK += dS^T Q_i and dQ_i = dS K_j, once dS^T is in shared memory
+                // dQ_i = dS K_j and dK += dS^T Q_i, once dS^T is in shared memory
                 if (!(ok = mbar_wait_bounded(smem_u32(&ctl->ds_full), ph, abort_flag, p.err, p.timeout_ns))) break;
                 tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kBwdKeys / 16; ++kk)
+                    tc_mma_ss(tDP, dS_mmaj + (uint64_t)((kk * 2048) >> 4), dK_nmaj + (uint64_t)((kk * 2048) >> 4),
+                              idesc_q, kk > 0 ? 1u : 0u);
+                tc_commit(smem_u32(&ctl->dq_full));  // dQ first: its read-out overlaps dK
 #pragma unroll
                 for (int kk = 0; kk < kBwdRows / 16; ++kk) {
                     const uint64_t ko = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
                     tc_mma_ss(tDK, dS_kmaj + ko, dQ_nmaj + (uint64_t)((kk * 2048) >> 4), idesc_kv,
                               (w > 0 || kk > 0) ? 1u : 0u);
                 }
-#pragma unroll
-                for (int kk = 0; kk < kBwdKeys / 16; ++kk)
-                    tc_mma_ss(tDP, dS_mmaj + (uint64_t)((kk * 2048) >> 4), dK_nmaj + (uint64_t)((kk * 2048) >> 4),
-                              idesc_q, kk > 0 ? 1u : 0u);
-                tc_commit(smem_u32(&ctl->dq_full));
                 tc_commit(smem_u32(&ctl->ds_empty));
                 tc_commit(smem_u32(&ctl->q_empty[slot]));
             }
