@@ -44,8 +44,7 @@ HostPlan plan_host(int B, int Hq, int Hkv, int Tq, int Tk, int D) {
     p.k_bytes = round_up256((size_t)B * Hkv * Tk * D * 2);
     p.q_slot_bytes = round_up256((size_t)B * Hq * rows * D * 2);
     p.lse_slot_bytes = round_up256((size_t)B * Hq * rows * sizeof(float));
-    size_t at = p.k_bytes;
-    p.off_v = 0;
+    size_t at = p.k_bytes;  // K first, then V
     p.off_v = at;
     at += p.k_bytes;
     for (int s = 0; s < 2; ++s) {
@@ -72,8 +71,8 @@ gqa_status check_host_args(const void* q, const void* k, const void* v, const vo
     return GQA_OK;
 }
 
-// Rows [r0, r1) of every (b, h) plane of a [planes, T, width] array: one 2-D copy whose
-// "rows" are the planes (pitch T * width bytes on the strided side).
+// A run of `bytes` bytes from each of `planes` (b, h) planes: one 2-D copy whose "rows" are
+// the planes, each side advancing by its own pitch from one plane to the next.
 cudaError_t copy_rows(void* dst, size_t dst_pitch, const void* src, size_t src_pitch, size_t bytes, size_t planes,
                       cudaMemcpyKind kind, cudaStream_t s) {
     return cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, bytes, planes, kind, s);
