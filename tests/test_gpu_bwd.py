@@ -55,6 +55,7 @@ CASES = [
     (2, 6, 2, 256, 256, 128),      # G = 3
     (1, 4, 4, 129, 257, 64),       # MHA, D = 64, suffix offset 128
     (1, 8, 2, 1000, 1000, 128),    # several tiles per key block and per query head
+    (3, 6, 2, 384, 384, 64),       # 6 (batch, KV head) pairs launched as one chunk, longest blocks first
 ]
 
 
