@@ -782,7 +782,8 @@ def main(argv=None):
         line["swa_prefill"] = {
             "metric": "TFLOP/s (window-visible pairs)", "value": throughput(ws_, mss, world),
             "unit": "TFLOP/s", "ms_per_step": mss, "config": workload_config(ws_),
-            "roofline": tensor_roofline(ach, peaks, peak_src, clocks, None, "gqa_fwd_sm100_kernel<window>"),
+            "roofline": tensor_roofline(ach, peaks, peak_src, clocks, load_traffic("gqa_fwd_sm100_kernel", ws_.name),
+                                        "gqa_fwd_sm100_kernel<window>"),
             "gpu_launches": rs["launches"]}
         wc = gi.WORKLOADS["chunk_decode"]
         nst = max(3, args.steps // 20)
@@ -793,7 +794,7 @@ def main(argv=None):
             "metric": "KV GB/s", "value": throughput(wc, msc, world), "unit": "GB/s", "ms_per_step": msc,
             "config": workload_config(wc, {"splits": rc_["splits"]}),
             "roofline": {"bound": "hbm", "achieved": achc, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achc / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achc / peaks["hbm_gbs"], "traffic": load_traffic("gqa_decode_sm100_kernel", wc.name),
                          "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
             "gpu_launches": rc_["launches"]}
         # variable-length rows: packed prefill, chunked prefill after cached prefixes,
