@@ -52,11 +52,16 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between
 // every kPolyEvery-th column pair of an unmasked tile takes the polynomial exp2 (0 = none)
 constexpr int kPolyEvery = GQA_FWD_POLY_EVERY;
 
+constexpr int kUnitPairHeads = 1;
+constexpr int kUnitHeadMajor = 2;
+
 struct FwdParams {
     int B, Hq, Hkv, Tq, Tk, G;
     int n_qt;        // ceil(Tq / 128)
-    int pair_heads;  // 1: sub-tiles are heads (a, a+1) of one group on the same rows
-                     // 0: sub-tiles are rows (r, r+128) of one head
+    int unit_flags;  // kUnitPairHeads: sub-tiles are heads (a, a+1) of one group on the same
+                     //   rows, else rows (r, r+128) of one head
+                     // kUnitHeadMajor: units listed head by head (all row levels of one head
+                     //   together), else level by level, longest rows first
     int per_level;   // work units per row level
     int units;       // total work units (grid-strided by the persistent CTAs)
     float scale_log2;
@@ -151,9 +156,18 @@ __device__ __forceinline__ void fwd_fill_subtile(SubTile& st, int len_q, int off
 __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& b, int& g,
                                                 SubTile (&st)[2]) {
     const int off = p.Tk - p.Tq;
-    const int level = u / p.per_level;
-    const int rest = u - level * p.per_level;
-    if (p.pair_heads) {
+    const bool pair = (p.unit_flags & kUnitPairHeads) != 0;
+    int level, rest;
+    if (p.unit_flags & kUnitHeadMajor) {
+        // the row levels of one head (pair) run side by side and share its K/V through L2
+        const int n_lvl = pair ? p.n_qt : (p.n_qt + 1) >> 1;
+        rest = u / n_lvl;
+        level = u - rest * n_lvl;
+    } else {
+        level = u / p.per_level;
+        rest = u - level * p.per_level;
+    }
+    if (pair) {
         const int half_g = p.G >> 1;
         const int rt = p.n_qt - 1 - level;  // longest rows first
         b = rest / (p.Hkv * half_g);
@@ -198,7 +212,7 @@ __device__ __forceinline__ void fwd_varlen_unit(const FwdParams& p, const FwdVar
     const int s = t / vp.n_lvl;
     fwd_seq_side(vp.cu_q, vp.len_q, vp.rows_q, s, geo.b_q, geo.r_q, geo.len_q);
     fwd_seq_side(vp.cu_k, vp.len_k, vp.rows_k, s, geo.b_k, geo.r_k, geo.len_k);
-    if (p.pair_heads) {
+    if (p.unit_flags & kUnitPairHeads) {
         st[0].head = 2 * hidx;
         st[1].head = 2 * hidx + 1;
         st[0].row0 = st[1].row0 = lvl * kFwdRows;

@@ -33,9 +33,13 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     p.Tk = a.Tk;
     p.G = a.Hq / a.Hkv;
     p.n_qt = (a.Tq + kFwdRows - 1) / kFwdRows;
-    p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+    p.unit_flags = (p.G % 2 == 0) ? kUnitPairHeads : 0;
+    // A suffix at least as long as its prefix has row levels of similar length, so units go
+    // head by head: the levels of one head then read its K/V from L2 rather than from HBM
+    // once per level (the K/V of all heads can exceed L2, as with many MHA heads)
+    if (a.Tk - a.Tq >= a.Tq) p.unit_flags |= kUnitHeadMajor;
     long long units;
-    if (p.pair_heads) {
+    if (p.unit_flags & kUnitPairHeads) {
         p.per_level = a.B * a.Hkv * (p.G / 2);
         units = (long long)p.per_level * p.n_qt;
     } else {
@@ -83,7 +87,7 @@ static cudaError_t launch_fwd_varlen_d(const FwdVarlenLaunch& a, cudaStream_t st
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
     p.G = a.Hq / a.Hkv;
-    p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+    p.unit_flags = (p.G % 2 == 0) ? kUnitPairHeads : 0;
     FwdVarlenParams vp{};
     const long long n_cand = fwd_varlen_candidates(a.S, a.Hq, a.Hkv, a.max_q, &vp.n_lvl, &vp.n_h);
     if (n_cand <= 0 || n_cand > 0x7fffffffLL) return cudaErrorInvalidValue;
