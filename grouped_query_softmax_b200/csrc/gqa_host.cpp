@@ -18,6 +18,7 @@
 #include <cstdint>
 
 #include "../../include/gqa.h"
+#include "../../include/gqa_testing.h"
 
 namespace {
 
@@ -59,6 +60,12 @@ HostPlan plan_host(int B, int Hq, int Hkv, int Tq, int Tk, int D) {
     return p;
 }
 
+// Query rows of chunk c (the last chunk may be shorter).
+int chunk_rows_of(const HostPlan& pl, int c, int Tq) {
+    const int r0 = c * pl.chunk_rows;
+    return (Tq - r0 < pl.chunk_rows) ? Tq - r0 : pl.chunk_rows;
+}
+
 gqa_status check_host_args(const void* q, const void* k, const void* v, const void* o, const float* lse, int B,
                            int Hq, int Hkv, int Tq, int Tk, int D, float scale, int window) {
     if (!q || !k || !v || !o) return GQA_ERR_INVALID_ARGUMENT;
@@ -86,6 +93,22 @@ size_t gqa_attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk,
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || (D != 64 && D != 128) || Hq % Hkv != 0 || Tq > Tk)
         return 0;
     return plan_host(B, Hq, Hkv, Tq, Tk, D).total;
+}
+
+gqa_status gqa_testing_fwd_host_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int* out_chunks, int* out_row0,
+                                     int* out_rows, int* out_keys) {
+    if (!out_chunks || !out_row0 || !out_rows || !out_keys) return GQA_ERR_INVALID_ARGUMENT;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || Hq % Hkv != 0 || Tq > Tk)
+        return GQA_ERR_INVALID_ARGUMENT;
+    if (D != 64 && D != 128) return GQA_ERR_INVALID_ARGUMENT;
+    const HostPlan pl = plan_host(B, Hq, Hkv, Tq, Tk, D);
+    *out_chunks = pl.chunks;
+    for (int c = 0; c < pl.chunks; ++c) {
+        out_row0[c] = c * pl.chunk_rows;
+        out_rows[c] = chunk_rows_of(pl, c, Tq);
+        out_keys[c] = Tk - Tq + out_row0[c] + out_rows[c];
+    }
+    return GQA_OK;
 }
 
 gqa_status gqa_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -133,7 +156,7 @@ gqa_status gqa_attn_fwd_host(const void* q, const void* k, const void* v, void* 
         for (int c = 0; c < pl.chunks; ++c) {
             const int slot = c & 1;
             const int r0 = c * pl.chunk_rows;
-            const int rows = (Tq - r0 < pl.chunk_rows) ? Tq - r0 : pl.chunk_rows;
+            const int rows = chunk_rows_of(pl, c, Tq);
             const int keys = off + r0 + rows;  // keys this chunk's last row sees
             uint8_t* q_slot = ws + pl.off_q[slot];
             uint8_t* o_slot = ws + pl.off_o[slot];

@@ -35,6 +35,17 @@ GQA_API gqa_status gqa_selftest_bounded_wait(unsigned long long timeout_ns, void
 GQA_API gqa_status gqa_testing_bwd_order(int n_kb, int n_bg, int G, int Tq, int D, int* out_chunk, int* out_bg,
                                          int* out_j);
 
+/*
+ * The chunk plan of gqa_attn_fwd_host, for host-side tests. For the given sizes writes
+ * *out_chunks (at most 8) and, for each chunk c, out_row0[c], out_rows[c] (its query rows are
+ * out_row0[c] .. out_row0[c] + out_rows[c] - 1) and out_keys[c] (the number of leading key
+ * rows its suffix call reads). The three arrays are caller-owned host memory of 8 ints each.
+ * Touches no GPU. Returns GQA_ERR_INVALID_ARGUMENT for sizes gqa_attn_fwd_host rejects or a
+ * null pointer.
+ */
+GQA_API gqa_status gqa_testing_fwd_host_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int* out_chunks,
+                                             int* out_row0, int* out_rows, int* out_keys);
+
 #ifdef __cplusplus
 }
 #endif
