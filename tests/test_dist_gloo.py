@@ -47,3 +47,48 @@ def test_two_gloo_ranks_take_the_max_time_and_aggregate_work():
     for rank, worst, one, agg in res:
         assert worst == 11.0
         assert agg == pytest.approx(2 * one)
+
+
+def _bench_rank(rank, world, port, q):
+    """One rank of bench.main with the GPU measurements faked and the process group on gloo."""
+    import contextlib
+    import io
+
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    from tests.test_bench_line import FAKES
+    torch.cuda.set_device = lambda *a, **k: None
+    real_init = dist.init_process_group
+    dist.init_process_group = lambda backend, timeout=None, device_id=None: real_init("gloo", timeout=timeout)
+    for name, fake in FAKES.items():
+        setattr(bench, name, fake)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.main(["--gpus", str(world), "--steps", "4", "--warmup", "3", "--no-extensions", "--no-decode"])
+    q.put((rank, out.getvalue()))
+
+
+def test_bench_line_over_two_gloo_ranks():
+    import json
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    outs = dict(q.get(timeout=10) for _ in range(2))
+    assert outs[1].strip() == ""  # only rank 0 prints
+    d = json.loads([l for l in outs[0].splitlines() if l.startswith("{")][-1])
+    import bench
+    w = bench.gi.WORKLOADS["gqa_prefill"]
+    per_rank = bench.algorithmic_flops(w) / (d["ms_per_step"] * 1e-3) / 1e12
+    assert d["n_gpus"] == 2 and d["scaling"] == "weak"
+    assert d["value"] == pytest.approx(2 * per_rank)
+    assert d["config"]["parallelism"].startswith("dp2")
+    assert "cpu_baseline" not in d  # the oracle baseline runs at one rank only
