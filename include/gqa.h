@@ -120,7 +120,10 @@ GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, 
  *            valid and unchanged until the stream gets there.
  *
  * Errors:
- *   - Argument errors are reported as for gqa_attn_fwd_ex, before anything is enqueued.
+ *   - Checked before anything is enqueued. GQA_ERR_INVALID_ARGUMENT for a null q, k, v or o,
+ *     a non-positive size, Hq % Hkv != 0, T_q > T_k, window < 0, an lse that is not 4-byte
+ *     aligned, or a non-finite scale. GQA_ERR_UNSUPPORTED for D outside {64, 128}. Host
+ *     pointers need no alignment.
  *   - A missing, misaligned or short workspace returns GQA_ERR_WORKSPACE.
  *   - GQA_ERR_CUDA means that a stream, event, copy or launch call failed. Part of the
  *     work may then already be enqueued: synchronise the device before reusing o or the
