@@ -1,15 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of causal grouped-query softmax attention on B200.
 
-One step = one pass of the hot path over one batch of synthetic input:
-  * headline: gqa_attn_fwd on the GQA prefill workload (B4 Hq32 Hkv8 T4096 D128),
-    metric TFLOP/s with FLOPs = 4 * D * Hq * B * (causal-visible query/key pairs);
-  * "decode" object: gqa_attn_decode on the GQA decode workload (B64 Hq32 Hkv8,
-    T_k 32768, D128), metric KV GB/s = (K + V bytes) / time.
-Inputs are seeded iid N(0,1) rounded to bf16 (see gqa_inputs), resident in HBM
-when the timed region starts. Under torchrun every rank runs its own copy of the
-workload (independent problems, no data-path collective): weak scaling, value =
-all ranks' work / max-over-ranks time.
+One step = one pass of the hot path over one batch of synthetic input. The main line is
+gqa_attn_fwd on the GQA prefill workload (B4 Hq32 Hkv8 T4096 D128), metric TFLOP/s with
+FLOPs = 4 * D * Hq * B * (causal-visible query/key pairs), timed over exactly --steps
+steps with inputs resident in HBM; a second pass of at least --long-pass seconds gives the
+clock record a long window; "e2e" is the host-memory call gqa_attn_fwd_host end to end.
+
+"rows" holds the other measurements, each its own step timed alone, the benchmark configs
+last: the extension workloads (sliding window, verify chunk, variable-length, paged,
+backward), then MQA long prefill (B1 Hq32 Hkv1 T32768), MHA suffix (B8 H16 Tq512 over
+Tk8192, Q x 4) and GQA decode (B64 Hq32 Hkv8 Tk32768; KV GB/s = (K + V bytes) / time),
+each of these three with the fp64 oracle's time on the host cores beside it.
+
+Inputs are seeded iid N(0,1) rounded to bf16 (see gqa_inputs). Under torchrun every rank
+runs its own copy of the workload (independent problems, no data-path collective): weak
+scaling, value = all ranks' work / max-over-ranks time.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of the
 method here) on a bounded row sample of the same workload, on the host cores.
@@ -34,6 +40,7 @@ import numpy as np  # noqa: E402
 
 import gqa_inputs as gi  # noqa: E402
 
+L2_NOTE = "inputs larger than L2 (no flush)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 _CSRC = "grouped_query_softmax_b200/csrc/"
 # The sources each kernel is compiled from: a traffic figure stays valid while these hash
@@ -89,27 +96,38 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def tensor_peak(peaks, peak_src, clocks):
-    """(peak, description): the sustained GEMM figure when the timed region ran at the power
-    cap, otherwise the burst figure."""
-    capped = "sw_power_cap" in (clocks.get("reasons") or [])
-    burst = peaks["bf16_tflops"]
-    if capped:
-        return (peaks.get("bf16_tflops_sustained", burst),
-                f"{peak_src} bf16_tflops_sustained (sw_power_cap active in the timed region)")
-    return burst, f"{peak_src} bf16_tflops (burst; kernel timed alone)"
+def tensor_peak(peaks, peak_src):
+    """(peak, description): every kernel here is timed alone, so the burst GEMM figure."""
+    return peaks["bf16_tflops"], f"{peak_src} bf16_tflops (burst; kernel timed alone)"
 
 
-def tensor_roofline(achieved, peaks, peak_src, clocks, traffic, kernel):
-    """The roofline object of a tensor-bound row: the power-cap-aware peak and the fraction
-    of it, with the fractions of the burst and sustained figures for context."""
-    peak, src = tensor_peak(peaks, peak_src, clocks)
-    burst = peaks["bf16_tflops"]
-    sustained = peaks.get("bf16_tflops_sustained", burst)
+def tensor_roofline(achieved, peaks, peak_src, traffic, kernel):
+    """The roofline object of a tensor-bound main line: the fraction of the burst peak,
+    with the fractions of the sustained (power-capped) and 2250 TFLOP/s spec figures for
+    context."""
+    peak, src = tensor_peak(peaks, peak_src)
+    sustained = peaks.get("bf16_tflops_sustained", peak)
     return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic, "peak_source": src,
-            "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
-            "frac_of_spec_2250": achieved / 2250.0, "kernel": kernel}
+            "frac_of_sustained": achieved / sustained, "frac_of_spec_2250": achieved / 2250.0, "kernel": kernel}
+
+
+def sig(x, n: int = 4):
+    """x to n significant digits (keeps the JSON line short); None stays None."""
+    return None if x is None else float(f"{x:.{n}g}")
+
+
+def row_entry(value, ms, achieved, peak, traffic, workload=None, cpu=None):
+    """One sub-row of the bench line: throughput, time per step and the roofline of its
+    dominant kernel (achieved / peak in the row's own unit; traffic = DRAM bytes per launch
+    from a committed ncu capture, or None)."""
+    r = {} if workload is None else {"workload": workload}
+    r.update({"value": sig(value), "ms_per_step": sig(ms),
+              "roofline": {"achieved": sig(achieved), "peak": peak, "frac": sig(achieved / peak),
+                           "traffic": traffic}})
+    if cpu is not None:
+        r["cpu_baseline"] = cpu
+    return r
 
 
 def load_peaks():
@@ -134,19 +152,63 @@ def load_traffic(kernel: str, workload: str):
 
 
 # ---------------------------------------------------------------- clocks
-class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons while the GPU is busy."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_id: str | None):
+
+class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled while it works.
+
+    NVML is polled every millisecond from a thread (its calls release the GIL), so even
+    a 10 ms timed region holds several samples; without NVML, nvidia-smi is sampled every
+    50 ms instead. Samples are (wall time, sm MHz, max sm MHz, set of active reasons)."""
+
+    def __init__(self, gpu_id: str | None, dev_index: int | None = None, interval_s: float = 0.001):
         self.samples = []
         self.proc = None
         self.gpu_id = gpu_id
+        self.dev_index = dev_index
+        self.interval_s = interval_s
+        self.source = "none"
+        self._stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:  # the CUDA device's own UUID is immune to CUDA_VISIBLE_DEVICES remapping
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev_index or 0).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id or 0))
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        try:
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            return self._start_smi()
+        self.source = f"nvml every {self.interval_s * 1e3:g} ms"
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    word = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                self.samples.append((time.time(), sm, smax, {n for n, b in bits.items() if word & b}))
+                time.sleep(self.interval_s)
+        threading.Thread(target=poll, daemon=True).start()
+
+    def _start_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        cmd = ["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.gpu_id is not None:
             cmd += ["-i", self.gpu_id]
         try:
@@ -154,15 +216,24 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
-        threading.Thread(target=self._reader, daemon=True).start()
+        self.source = "nvidia-smi every 50 ms"
 
-    def _reader(self):
-        for line in self.proc.stdout:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append((time.time(), parts))
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        def read():
+            for line in self.proc.stdout:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 6:
+                    active = {REASON_NAMES[i] for i in range(4) if parts[2 + i].lower().startswith("active")}
+                    self.samples.append((time.time(), num(parts[0]), num(parts[1]), active))
+        threading.Thread(target=read, daemon=True).start()
 
     def stop(self):
+        self._stop.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -171,24 +242,29 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0: float, t1: float):
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        window = [s for t, s in self.samples if t0 <= t <= t1]
+        """Median SM clock and every reason seen between t0 and t1 (wall time)."""
+        window = [s for s in self.samples if t0 <= s[0] <= t1]
         scope = "timed region"
         if len(window) < 3:
-            window = [s for _, s in self.samples]
+            window = list(self.samples)
             scope = "whole run (timed region shorter than the sampling interval)"
         if not window:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "scope": "unavailable"}
-        sm = [num(s[1]) for s in window if num(s[1]) is not None]
-        smax = [num(s[2]) for s in window if num(s[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in window for i in range(4) if s[5 + i].lower().startswith("active")})
+        sm = [s[1] for s in window if s[1] is not None]
+        smax = [s[2] for s in window if s[2] is not None]
+        reasons = sorted(set().union(*(s[3] for s in window)))
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(window), "scope": scope}
+                "reasons": reasons, "samples": len(window), "scope": scope, "source": self.source}
+
+
+def make_sampler(local: int, world: int) -> ClockSampler:
+    """A started sampler for this rank's GPU (CUDA device `local`)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = vis.split(",")[local] if vis else str(local)
+    s = ClockSampler(gpu_id, local)
+    s.start()
+    time.sleep(0.2)
+    return s
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -245,23 +321,39 @@ def timed(fn, steps, warmup, world, dev):
     return max_over_ranks(ms, world, dev), t0, t1
 
 
-def measure_prefill(w, steps, warmup, world, dev, e2e_steps):
+def long_pass(fn, res, long_s, world, dev):
+    """A second timed pass of the same step lasting at least long_s seconds, so the clock
+    sampler sees it; its step count follows from the first pass (the same on every rank)."""
+    if long_s <= 0:
+        return
+    ms_step = res["ms_total"] / res["steps"]
+    n = max(res["steps"], int(math.ceil(long_s * 1e3 / max(ms_step, 1e-6))))
+    ms, t0, t1 = timed(fn, n, 0, world, dev)
+    res.update(long_steps=n, long_ms_total=ms, long_t0=t0, long_t1=t1)
+
+
+def measure_prefill(w, steps, warmup, world, dev, e2e_steps=0, inputs=None, long_s=0.0):
+    """gqa_attn_fwd over `steps` calls on inputs resident in HBM; optionally a long pass of
+    the same call, and the host-memory call end to end (e2e_steps > 0)."""
     import torch
     import grouped_query_softmax_b200 as gqa
-    q, k, v = w.make()
+    q, k, v = inputs if inputs is not None else w.make()
     qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
     od = torch.empty_like(qd)
     fn = lambda: gqa.attn_fwd(qd, kd, vd, out=od, window=w.window)
     ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": steps, "steps": steps}
+    long_pass(fn, res, long_s, world, dev)
     st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
     if st != gqa.GQA_OK:
         raise RuntimeError(f"device error after prefill timing: {gqa.gqa_status_string(st)}")
-    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": steps}
+    del qd, kd, vd, od
+    torch.cuda.empty_cache()
+    if e2e_steps <= 0:
+        return res
 
     # end to end through the public host-memory call (gqa_attn_fwd_host): pinned host inputs
     # in, host output out, every step; its device workspace is allocated once, outside
-    del qd, kd, vd, od
-    torch.cuda.empty_cache()
     qh = torch.from_numpy(q.view(np.int16)).pin_memory().view(torch.bfloat16)
     kh = torch.from_numpy(k.view(np.int16)).pin_memory().view(torch.bfloat16)
     vh = torch.from_numpy(v.view(np.int16)).pin_memory().view(torch.bfloat16)
@@ -280,10 +372,12 @@ def measure_prefill(w, steps, warmup, world, dev, e2e_steps):
     return res
 
 
-def measure_decode(w, steps, warmup, world, dev, e2e_steps):
+def measure_decode(w, steps, warmup, world, dev, e2e_steps=0, inputs=None, long_s=0.0):
+    """gqa_attn_decode(_ex) over `steps` calls on a cache resident in HBM; optionally a long
+    pass, and end to end with the inputs copied from pinned host memory every step."""
     import torch
     import grouped_query_softmax_b200 as gqa
-    q, k, v = w.make()
+    q, k, v = inputs if inputs is not None else w.make()
     qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
     od = torch.empty_like(qd)
     splits = gqa.gqa_attn_decode_ex_num_splits(w.B, w.Hq, w.Hkv, w.Tq, w.Tk, w.D, w.window, 0)
@@ -291,26 +385,28 @@ def measure_decode(w, steps, warmup, world, dev, e2e_steps):
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     fn = lambda: gqa.attn_decode(qd, kd, vd, out=od, workspace=ws, window=w.window)
     ms, t0, t1 = timed(fn, steps, warmup, world, dev)
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "splits": splits, "steps": steps,
+           "launches": steps * (1 if splits == 1 else 2)}
+    long_pass(fn, res, long_s, world, dev)
     st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
     if st != gqa.GQA_OK:
         raise RuntimeError(f"device error after decode timing: {gqa.gqa_status_string(st)}")
-    res = {"ms_total": ms, "t0": t0, "t1": t1, "splits": splits,
-           "launches": steps * (1 if splits == 1 else 2)}
-    qh = torch.from_numpy(q.view(np.int16)).pin_memory()
-    kh = torch.from_numpy(k.view(np.int16)).pin_memory()
-    vh = torch.from_numpy(v.view(np.int16)).pin_memory()
-    oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
-    qi, ki, vi, oi = (x.view(torch.int16) for x in (qd, kd, vd, od))
+    if e2e_steps > 0:
+        qh = torch.from_numpy(q.view(np.int16)).pin_memory()
+        kh = torch.from_numpy(k.view(np.int16)).pin_memory()
+        vh = torch.from_numpy(v.view(np.int16)).pin_memory()
+        oh = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+        qi, ki, vi, oi = (x.view(torch.int16) for x in (qd, kd, vd, od))
 
-    def e2e_step():
-        qi.copy_(qh, non_blocking=True)
-        ki.copy_(kh, non_blocking=True)
-        vi.copy_(vh, non_blocking=True)
-        gqa.attn_decode(qd, kd, vd, out=od, workspace=ws, window=w.window)
-        oh.copy_(oi, non_blocking=True)
-    e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
-    res.update(e2e_ms_total=e2e_ms, e2e_steps=e2e_steps, h2d_bytes=int(q.nbytes + k.nbytes + v.nbytes),
-               d2h_bytes=int(q.nbytes))
+        def e2e_step():
+            qi.copy_(qh, non_blocking=True)
+            ki.copy_(kh, non_blocking=True)
+            vi.copy_(vh, non_blocking=True)
+            gqa.attn_decode(qd, kd, vd, out=od, workspace=ws, window=w.window)
+            oh.copy_(oi, non_blocking=True)
+        e2e_ms, _, _ = timed(e2e_step, e2e_steps, 1, world, dev)
+        res.update(e2e_ms_total=e2e_ms, e2e_steps=e2e_steps, h2d_bytes=int(q.nbytes + k.nbytes + v.nbytes),
+                   d2h_bytes=int(q.nbytes))
     del qd, kd, vd, od, ws
     torch.cuda.empty_cache()
     return res
@@ -511,6 +607,25 @@ def oracle_sample(w, budget_s: float, threads: int, q=None, k=None, v=None):
     return row_flops(w, rows), dt, rows
 
 
+def oracle_baseline(w, budget_s: float, threads: int, inputs=None):
+    """The fp64 oracle on the host cores, on workload w: every output row when that takes
+    about budget_s seconds or less, else a seeded row sample whose time is extrapolated to
+    the whole workload by visible pairs (and labelled so). A reported baseline."""
+    q, k, v = inputs if inputs is not None else w.make()
+    flops, secs, rows = oracle_sample(w, budget_s, threads, q, k, v)
+    total = w.B * w.Hq * w.Tq
+    if is_decode(w):
+        value, unit = len(rows) / total * kv_bytes(w) / secs / 1e9, "GB/s"
+    else:
+        value, unit = flops / secs / 1e12, "TFLOP/s"
+    if len(rows) >= total:
+        sample = f"all {total} output rows (fp64), {secs:.1f} s"
+    else:
+        sample = (f"{len(rows)} of {total} output rows (seeded sample, fp64), {secs:.1f} s; "
+                  f"full run extrapolated by visible pairs: {secs * algorithmic_flops(w) / flops:.0f} s")
+    return {"value": sig(value), "unit": unit, "cores": threads, "kind": "oracle", "sample": sample}
+
+
 def cpu_threads() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -527,14 +642,16 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gqa_prefill", choices=sorted(gi.WORKLOADS) + sorted(gi.VARLEN_WORKLOADS),
                     help="main workload (a varlen or paged one is measured alone, e.g. for profiling)")
-    ap.add_argument("--decode-workload", default="gqa_decode", choices=sorted(gi.WORKLOADS))
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the rows of the other benchmark configs (MQA long, MHA suffix, GQA decode)")
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the sliding-window, decode-chunk and variable-length measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--backward", action="store_true",
                     help="measure only the backward pass of the main (dense) workload, e.g. for profiling")
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work on the main workload")
+    ap.add_argument("--long-pass", type=float, default=1.0,
+                    help="seconds of a second timed pass of the main step, long enough for the clock record")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--batch", type=int, default=0,
                     help="override the main workload's batch size / sequence count (for profiling a smaller case)")
@@ -542,8 +659,9 @@ def parse_args(argv=None):
 
 
 def workload_config(w, extra=None):
+    """The config object of a dense workload; both bench arms print the same one."""
     c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Tq": w.Tq, "Tk": w.Tk, "D": w.D,
-         "q_scale": 2 ** w.q_pow2, "seed": w.seed, "causal": True}
+         "q_scale": 2 ** w.q_pow2, "seed": w.seed, "causal": True, "l2": L2_NOTE}
     if w.window:
         c["window"] = w.window
     if extra:
@@ -601,9 +719,7 @@ def reference_arm(args, rank, world):
 
 def backward_main(args, rank, world, local, dev, peaks, peak_src, w):
     """The backward pass of a dense workload as the main line (profiling and focused runs)."""
-    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local])
-    sampler.start()
-    time.sleep(0.2)
+    sampler = make_sampler(local, world)
     r = measure_bwd(w, args.steps, args.warmup, world, dev)
     ms_step = r["ms_total"] / args.steps
     achieved = bwd_flops(w) / (ms_step * 1e-3) / 1e12
@@ -612,10 +728,8 @@ def backward_main(args, rank, world, local, dev, peaks, peak_src, w):
     line = {"metric": "GQA attn backward TFLOP/s on 1 B200, % of roofline", "value": world * achieved,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, {"pass": "backward (dQ, dK, dV)", "l2": "inputs larger than L2 (no flush)",
-                                          "parallelism": f"dp{world} (independent problems per rank)"}),
-            "roofline": tensor_roofline(achieved, peaks, peak_src, clocks,
-                                        load_traffic("gqa_bwd_sm100_kernel", w.name),
+            "config": workload_config(w, {"pass": "backward (dQ, dK, dV)"}),
+            "roofline": tensor_roofline(achieved, peaks, peak_src, load_traffic("gqa_bwd_sm100_kernel", w.name),
                                         "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"),
             "gpu_launches": r["launches"], "clocks": clocks}
     if world > 1:
@@ -633,9 +747,7 @@ def varlen_main(args, rank, world, local, dev, peaks, peak_src):
     if args.batch > 0:
         field = "B" if isinstance(w, gi.PagedDecodeWorkload) else "S"
         w = dataclasses.replace(w, **{field: args.batch}, name=f"{w.name} ({field} {args.batch})")
-    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local])
-    sampler.start()
-    time.sleep(0.2)
+    sampler = make_sampler(local, world)
     if isinstance(w, gi.PagedDecodeWorkload):
         r = measure_paged_decode(w, args.steps, args.warmup, world, dev, args.e2e_steps)
         work, unit, scale = paged_kv_bytes(w), "GB/s", 1e9
@@ -656,8 +768,8 @@ def varlen_main(args, rank, world, local, dev, peaks, peak_src):
     clocks = sampler.summary(r["t0"], r["t1"])
     sampler.stop()
     if bound == "tensor":
-        roof = tensor_roofline(achieved, peaks, peak_src, clocks,
-                               load_traffic("gqa_fwd_sm100_kernel_varlen", w.name), kernel)
+        roof = tensor_roofline(achieved, peaks, peak_src, load_traffic("gqa_fwd_sm100_kernel_varlen", w.name),
+                               kernel)
     else:
         roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": load_traffic("gqa_decode_sm100_kernel_varlen", w.name), "peak_source": src,
@@ -665,8 +777,7 @@ def varlen_main(args, rank, world, local, dev, peaks, peak_src):
     line = {"metric": metric, "value": world * achieved, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config | {"l2": "inputs larger than L2 (no flush)",
-                                "parallelism": f"dp{world} (independent problems per rank)"},
+            "config": config | {"l2": L2_NOTE},
             "roofline": roof,
             "gpu_launches": r["launches"], "clocks": clocks}
     if args.e2e_steps:
@@ -680,6 +791,93 @@ def varlen_main(args, rank, world, local, dev, peaks, peak_src):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# The other benchmark configs, measured as rows of the default line (last in it), each with
+# the oracle's time on the host cores beside it: (key, workload, oracle seconds).
+CONFIG_ROWS = (("mqa_long", "mqa_long", 5.0), ("mha_suffix", "mha_suffix", 8.0), ("decode", "gqa_decode", 3.0))
+
+
+def hbm_row(work_bytes, ms, peaks, traffic, workload=None, cpu=None, world=1):
+    gbs = work_bytes / (ms * 1e-3) / 1e9
+    return row_entry(world * gbs, ms, gbs, peaks["hbm_gbs"], traffic, workload, cpu)
+
+
+def tensor_row(flops, ms, peaks, traffic, workload=None, cpu=None, world=1):
+    tf = flops / (ms * 1e-3) / 1e12
+    return row_entry(world * tf, ms, tf, peaks["bf16_tflops"], traffic, workload, cpu)
+
+
+def extension_rows(args, w, world, dev, peaks):
+    """The rows of the extension workloads: sliding window, verify chunk, variable-length,
+    paged and backward (each its own step, timed alone)."""
+    rows = {}
+    warm = max(3, args.warmup)
+    nsv = max(10, args.steps // 4)   # prefill-sized rows
+    nsd = max(3, args.steps // 20)   # decode-sized rows (8 GB of cache per step)
+    ws_ = gi.WORKLOADS["swa_prefill"]
+    r = measure_prefill(ws_, nsv, warm, world, dev)
+    rows["swa_prefill"] = tensor_row(algorithmic_flops(ws_), r["ms_total"] / nsv, peaks,
+                                     load_traffic("gqa_fwd_sm100_kernel", ws_.name), world=world)
+    wc = gi.WORKLOADS["chunk_decode"]
+    r = measure_decode(wc, nsd, warm, world, dev)
+    rows["chunk_decode"] = hbm_row(kv_bytes(wc) + qo_bytes(wc), r["ms_total"] / nsd, peaks,
+                                   load_traffic("gqa_decode_sm100_kernel", wc.name), world=world)
+    for key in ("varlen_prefill", "chunked_prefill"):
+        wv = gi.VARLEN_WORKLOADS[key]
+        r = measure_varlen(wv, nsv, warm, world, dev)
+        rows[key] = tensor_row(varlen_flops(wv), r["ms_total"] / nsv, peaks,
+                               load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name), world=world)
+    # the chunked-prefill workload again, its keys read from a paged pool of 64-key pages
+    wv = gi.VARLEN_WORKLOADS["chunked_prefill"]
+    r = measure_paged_prefill(wv, 64, nsv, warm, world, dev)
+    rows["paged_chunked_prefill"] = tensor_row(varlen_flops(wv), r["ms_total"] / nsv, peaks, None, world=world)
+    wp = gi.VARLEN_WORKLOADS["paged_decode"]
+    r = measure_paged_decode(wp, nsd, warm, world, dev)
+    rows["paged_decode"] = hbm_row(paged_kv_bytes(wp), r["ms_total"] / nsd, peaks,
+                                   load_traffic("gqa_decode_sm100_kernel_varlen", wp.name), world=world)
+    # backward (dQ, dK, dV) of the GQA prefill workload
+    r = measure_bwd(w, nsv, warm, world, dev)
+    rows["backward"] = tensor_row(bwd_flops(w), r["ms_total"] / nsv, peaks,
+                                  load_traffic("gqa_bwd_sm100_kernel", w.name), world=world)
+    return rows
+
+
+def make_inputs(w):
+    """Host (q, k, v) bf16 bit arrays of a dense workload, shared by the GPU row and the oracle."""
+    return w.make()
+
+
+def config_rows(args, w, world, dev, peaks, with_cpu):
+    """The benchmark configs other than the main one (MQA long, MHA suffix, GQA decode),
+    each with the oracle beside it on rank 0 at N = 1."""
+    rows = {}
+    threads = cpu_threads()
+    for key, name, budget in CONFIG_ROWS:
+        wr = gi.WORKLOADS[name]
+        if wr.name == w.name:
+            continue
+        inputs = make_inputs(wr)
+        if is_decode(wr):
+            n = max(3, args.steps // 20)
+            r = measure_decode(wr, n, max(3, args.warmup), world, dev, inputs=inputs)
+        else:
+            n = max(10, args.steps // 4)
+            r = measure_prefill(wr, n, max(3, args.warmup), world, dev, inputs=inputs)
+        cpu = oracle_baseline(wr, budget, threads, inputs) if with_cpu else None
+        del inputs
+        ms = r["ms_total"] / n
+        if is_decode(wr):
+            rows[key] = hbm_row(kv_bytes(wr) + qo_bytes(wr), ms, peaks,
+                                load_traffic("gqa_decode_sm100_kernel", wr.name), wr.name, cpu, world)
+        else:
+            rows[key] = tensor_row(algorithmic_flops(wr), ms, peaks,
+                                   load_traffic("gqa_fwd_sm100_kernel", wr.name), wr.name, cpu, world)
+    return rows
+
+
+def short_clocks(c):
+    return {k: c.get(k) for k in ("sm_mhz", "reasons", "samples", "scope")}
 
 
 def main(argv=None):
@@ -709,29 +907,17 @@ def main(argv=None):
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name} (batch {args.batch})")
     if args.backward:
         return backward_main(args, rank, world, local, dev, peaks, peak_src, w)
-    gpu_id = None
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        gpu_id = vis.split(",")[local]
-    elif world > 1:
-        gpu_id = str(local)
-    sampler = ClockSampler(gpu_id if gpu_id is not None else "0")
-    sampler.start()
-    time.sleep(0.2)
+    sampler = make_sampler(local, world)
 
     metric, unit = metric_of(w)
-    if is_decode(w):
-        r = measure_decode(w, args.steps, args.warmup, world, dev, args.e2e_steps)
-    else:
-        r = measure_prefill(w, args.steps, args.warmup, world, dev, args.e2e_steps)
+    measure = measure_decode if is_decode(w) else measure_prefill
+    r = measure(w, args.steps, args.warmup, world, dev, args.e2e_steps, long_s=args.long_pass)
     ms_step = r["ms_total"] / args.steps
     value = throughput(w, ms_step, world)
-    e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
     clocks = sampler.summary(r["t0"], r["t1"])
 
     if is_decode(w):
-        per_launch_bytes = kv_bytes(w) + qo_bytes(w)
-        achieved = per_launch_bytes / (ms_step * 1e-3) / 1e9
+        achieved = (kv_bytes(w) + qo_bytes(w)) / (ms_step * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": load_traffic("gqa_decode_sm100_kernel", w.name),
@@ -739,131 +925,37 @@ def main(argv=None):
                 "kernel": "gqa_decode_sm100_kernel + gqa_decode_combine_kernel (one call per step)"}
     else:
         achieved = algorithmic_flops(w) / (ms_step * 1e-3) / 1e12
-        roof = tensor_roofline(achieved, peaks, peak_src, clocks,
-                               load_traffic("gqa_fwd_sm100_kernel", w.name), "gqa_fwd_sm100_kernel")
+        roof = tensor_roofline(achieved, peaks, peak_src, load_traffic("gqa_fwd_sm100_kernel", w.name),
+                               "gqa_fwd_sm100_kernel")
 
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, {"l2": "inputs larger than L2 (no flush)",
-                                          "parallelism": f"dp{world} (independent problems per rank)"}),
-            "roofline": roof,
-            "e2e": {"value": throughput(w, e2e_ms, world), "unit": unit,
-                    "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"],
-                    "ms_per_step": e2e_ms, "steps": r["e2e_steps"],
-                    "call": ("gqa_attn_decode_ex after host-to-device copies of q, k, v" if is_decode(w) else
-                             "gqa_attn_fwd_host: pinned host q, k, v, o; query-row chunks overlap copies "
-                             "and kernels")},
-            "gpu_launches": r["launches"], "clocks": clocks}
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "roofline": roof, "gpu_launches": r["launches"], "clocks": clocks}
+    if args.e2e_steps > 0:
+        e2e_ms = r["e2e_ms_total"] / r["e2e_steps"]
+        line["e2e"] = {"value": throughput(w, e2e_ms, world), "unit": unit, "h2d_bytes_per_step": r["h2d_bytes"],
+                       "d2h_bytes_per_step": r["d2h_bytes"], "ms_per_step": e2e_ms, "steps": r["e2e_steps"],
+                       "call": ("gqa_attn_decode_ex after host-to-device copies of q, k, v" if is_decode(w) else
+                                "gqa_attn_fwd_host: pinned host q, k, v, o; query-row chunks overlap copies "
+                                "and kernels")}
+    if "long_steps" in r:
+        lms = r["long_ms_total"] / r["long_steps"]
+        line["long_pass"] = {"steps": r["long_steps"], "ms_per_step": lms, "value": throughput(w, lms, world),
+                             "clocks": short_clocks(sampler.summary(r["long_t0"], r["long_t1"]))}
 
-    if not args.no_decode and not is_decode(w):
-        wd = gi.WORKLOADS[args.decode_workload]
-        rd = measure_decode(wd, max(3, args.steps // 20), max(3, args.warmup), world, dev,
-                            max(2, args.e2e_steps // 5))
-        msd = rd["ms_total"] / max(3, args.steps // 20)
-        gbs = throughput(wd, msd, world)
-        ach = (kv_bytes(wd) + qo_bytes(wd)) / (msd * 1e-3) / 1e9
-        line["decode"] = {
-            "metric": "KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": msd,
-            "steps": max(3, args.steps // 20), "config": workload_config(wd, {"splits": rd["splits"]}),
-            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": ach / peaks["hbm_gbs"],
-                         "traffic": load_traffic("gqa_decode_sm100_kernel", wd.name),
-                         "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
-            "e2e": {"value": throughput(wd, rd["e2e_ms_total"] / rd["e2e_steps"], world), "unit": "GB/s",
-                    "h2d_bytes_per_step": rd["h2d_bytes"], "d2h_bytes_per_step": rd["d2h_bytes"]},
-            "gpu_launches": rd["launches"]}
-    if not args.no_extensions and not is_decode(w) and w.name == gi.GQA_PREFILL.name:
-        # the extension rows: sliding-window prefill and short decode chunks
-        ws_ = gi.WORKLOADS["swa_prefill"]
-        rs = measure_prefill(ws_, max(10, args.steps // 4), max(3, args.warmup), world, dev, 2)
-        mss = rs["ms_total"] / max(10, args.steps // 4)
-        ach = algorithmic_flops(ws_) / (mss * 1e-3) / 1e12
-        line["swa_prefill"] = {
-            "metric": "TFLOP/s (window-visible pairs)", "value": throughput(ws_, mss, world),
-            "unit": "TFLOP/s", "ms_per_step": mss, "config": workload_config(ws_),
-            "roofline": tensor_roofline(ach, peaks, peak_src, clocks, load_traffic("gqa_fwd_sm100_kernel", ws_.name),
-                                        "gqa_fwd_sm100_kernel<window>"),
-            "gpu_launches": rs["launches"]}
-        wc = gi.WORKLOADS["chunk_decode"]
-        nst = max(3, args.steps // 20)
-        rc_ = measure_decode(wc, nst, max(3, args.warmup), world, dev, 2)
-        msc = rc_["ms_total"] / nst
-        achc = (kv_bytes(wc) + qo_bytes(wc)) / (msc * 1e-3) / 1e9
-        line["chunk_decode"] = {
-            "metric": "KV GB/s", "value": throughput(wc, msc, world), "unit": "GB/s", "ms_per_step": msc,
-            "config": workload_config(wc, {"splits": rc_["splits"]}),
-            "roofline": {"bound": "hbm", "achieved": achc, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achc / peaks["hbm_gbs"], "traffic": load_traffic("gqa_decode_sm100_kernel", wc.name),
-                         "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
-            "gpu_launches": rc_["launches"]}
-        # variable-length rows: packed prefill, chunked prefill after cached prefixes,
-        # paged decode with per-sequence lengths
-        nsv = max(10, args.steps // 4)
-        for key in ("varlen_prefill", "chunked_prefill"):
-            wv = gi.VARLEN_WORKLOADS[key]
-            rv = measure_varlen(wv, nsv, max(3, args.warmup), world, dev)
-            msv = rv["ms_total"] / nsv
-            achv = varlen_flops(wv) / (msv * 1e-3) / 1e12
-            line[key] = {
-                "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achv,
-                "unit": "TFLOP/s", "ms_per_step": msv,
-                "config": varlen_config(wv) | {"tokens_q": rv["tokens_q"], "tokens_k": rv["tokens_k"]},
-                "roofline": tensor_roofline(achv, peaks, peak_src, clocks,
-                                            load_traffic("gqa_fwd_sm100_kernel_varlen", wv.name),
-                                            "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen>"),
-                "gpu_launches": rv["launches"]}
-        # the chunked-prefill workload again, its keys read from a paged pool
-        wv = gi.VARLEN_WORKLOADS["chunked_prefill"]
-        rpp = measure_paged_prefill(wv, 64, nsv, max(3, args.warmup), world, dev)
-        mspp = rpp["ms_total"] / nsv
-        achpp = varlen_flops(wv) / (mspp * 1e-3) / 1e12
-        line["paged_chunked_prefill"] = {
-            "metric": "TFLOP/s (causal-visible pairs of every sequence)", "value": world * achpp, "unit": "TFLOP/s",
-            "ms_per_step": mspp, "config": varlen_config(wv) | {"keys": "paged, 64 per page, seeded random page order"},
-            "roofline": tensor_roofline(achpp, peaks, peak_src, clocks, None,
-                                        "gqa_varlen_plan_kernel + gqa_fwd_sm100_kernel<varlen, paged>"),
-            "gpu_launches": rpp["launches"]}
-        # backward (training) on the headline workload
-        nsb = max(10, args.steps // 4)
-        rb = measure_bwd(w, nsb, max(3, args.warmup), world, dev)
-        msb = rb["ms_total"] / nsb
-        achb = bwd_flops(w) / (msb * 1e-3) / 1e12
-        line["backward"] = {
-            "metric": "TFLOP/s (10 * D * Hq * B * causal-visible pairs: S, dP, dV, dK, dQ)", "value": world * achb,
-            "unit": "TFLOP/s", "ms_per_step": msb, "config": workload_config(w),
-            "roofline": tensor_roofline(achb, peaks, peak_src, clocks,
-                                        load_traffic("gqa_bwd_sm100_kernel", w.name),
-                                        "gqa_bwd_prep_kernel + gqa_bwd_sm100_kernel + gqa_bwd_dq_kernel"),
-            "gpu_launches": rb["launches"]}
-        wp = gi.VARLEN_WORKLOADS["paged_decode"]
-        nsp = max(3, args.steps // 20)
-        rp = measure_paged_decode(wp, nsp, max(3, args.warmup), world, dev)
-        msp = rp["ms_total"] / nsp
-        achp = paged_kv_bytes(wp) / (msp * 1e-3) / 1e9
-        line["paged_decode"] = {
-            "metric": "KV GB/s (every cached key of every sequence)", "value": world * achp, "unit": "GB/s",
-            "ms_per_step": msp,
-            "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "D": wp.D, "Tq": wp.Tq,
-                       "cache_len": f"U[{wp.len_lo},{wp.len_hi}]", "page": wp.page,
-                       "pool": "[pages, page, Hkv, D], seeded random page order", "splits": rp["splits"]},
-            "roofline": {"bound": "hbm", "achieved": achp, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achp / peaks["hbm_gbs"],
-                         "traffic": load_traffic("gqa_decode_sm100_kernel_varlen", wp.name),
-                         "peak_source": f"{peak_src} hbm_gbs (copy, read+write bytes)"},
-            "gpu_launches": rp["launches"]}
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu
+    rows = {}
+    if not args.no_extensions and w.name == gi.GQA_PREFILL.name:
+        rows.update(extension_rows(args, w, world, dev, peaks))
+    if not args.no_configs:
+        rows.update(config_rows(args, w, world, dev, peaks, with_cpu))
     sampler.stop()
 
-    if rank == 0 and world == 1 and not args.no_cpu:
-        threads = cpu_threads()
-        flops, secs, rows = oracle_sample(w, args.cpu_budget, threads)
-        if is_decode(w):
-            cv = len(rows) / (w.B * w.Hq * w.Tq) * kv_bytes(w) / secs / 1e9
-        else:
-            cv = flops / secs / 1e12
-        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": threads, "kind": "oracle",
-                                "sample": f"{len(rows)} of {w.B * w.Hq * w.Tq} output rows "
-                                          f"(seeded sample, fp64), {secs:.1f} s"}
+    if with_cpu:
+        line["cpu_baseline"] = oracle_baseline(w, args.cpu_budget, cpu_threads())
+    if rows:
+        line["rows"] = rows
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -37,12 +37,10 @@ def test_flop_and_byte_counts():
     assert bench.paged_kv_bytes(pw) == 2 * int(pw.lengths().sum()) * pw.Hkv * pw.D * 2
 
 
-def test_tensor_peak_follows_the_power_cap():
+def test_tensor_peak_is_the_burst_figure():
     peaks = {"bf16_tflops": 1630.1, "bf16_tflops_sustained": 1374.1}
-    assert bench.tensor_peak(peaks, "measured", {"reasons": []})[0] == 1630.1
-    assert bench.tensor_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})[0] == 1374.1
-    assert "sustained" in bench.tensor_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})[1]
-    assert bench.tensor_peak({"bf16_tflops": 1590.0}, "fallback", {"reasons": ["sw_power_cap"]})[0] == 1590.0
+    assert bench.tensor_peak(peaks, "measured") == (1630.1, "measured bf16_tflops (burst; kernel timed alone)")
+    assert bench.tensor_peak({"bf16_tflops": 1590.0}, "fallback")[0] == 1590.0
 
 
 def test_traffic_figures_follow_their_kernel_sources():
@@ -62,11 +60,31 @@ def test_traffic_figures_follow_their_kernel_sources():
 
 def test_tensor_roofline_fractions():
     peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
-    r = bench.tensor_roofline(700.0, peaks, "measured", {"reasons": ["sw_power_cap"]}, 123, "k")
-    assert r["peak"] == 1400.0 and r["frac"] == 0.5 and r["frac_of_burst"] == 700.0 / 1600.0
-    assert r["traffic"] == 123 and r["kernel"] == "k" and r["bound"] == "tensor"
-    r = bench.tensor_roofline(800.0, peaks, "measured", {"reasons": []}, None, "k")
+    r = bench.tensor_roofline(800.0, peaks, "measured", 123, "k")
     assert r["peak"] == 1600.0 and r["frac"] == 0.5 and r["frac_of_sustained"] == 800.0 / 1400.0
+    assert r["traffic"] == 123 and r["kernel"] == "k" and r["bound"] == "tensor"
+
+
+def test_rows_round_to_four_digits():
+    r = bench.row_entry(1234.5678, 0.123456, 1234.5678, 1630.1, None, "w", {"value": 1})
+    assert r == {"workload": "w", "value": 1235.0, "ms_per_step": 0.1235,
+                 "roofline": {"achieved": 1235.0, "peak": 1630.1, "frac": 0.7574, "traffic": None},
+                 "cpu_baseline": {"value": 1}}
+    assert bench.sig(None) is None and bench.sig(0.000123456) == 0.0001235
+
+
+def test_oracle_baseline_full_and_extrapolated():
+    """All rows when the budget allows; otherwise a sample whose full-run time is
+    extrapolated by visible pairs, and labelled so."""
+    import dataclasses
+    w = gi.TINY
+    full = bench.oracle_baseline(w, 30.0, 2)
+    assert full["sample"].startswith(f"all {w.B * w.Hq * w.Tq} output rows") and full["value"] > 0
+    big = dataclasses.replace(w, Tq=4096, Tk=4096, name="tiny shape, long rows")
+    part = bench.oracle_baseline(big, 0.05, 2)
+    assert "extrapolated by visible pairs" in part["sample"] and part["unit"] == "TFLOP/s"
+    dec = dataclasses.replace(w, Tq=1, Tk=2048, name="tiny decode")
+    assert bench.oracle_baseline(dec, 10.0, 2)["unit"] == "GB/s"
 
 
 def _undefined_globals(path):

@@ -65,9 +65,10 @@ def _bench_rank(rank, world, port, q):
     dist.init_process_group = lambda backend, timeout=None, device_id=None: real_init("gloo", timeout=timeout)
     for name, fake in FAKES.items():
         setattr(bench, name, fake)
+    bench.make_inputs = lambda w: (None, None, None)
     out = io.StringIO()
     with contextlib.redirect_stdout(out):
-        bench.main(["--gpus", str(world), "--steps", "4", "--warmup", "3", "--no-extensions", "--no-decode"])
+        bench.main(["--gpus", str(world), "--steps", "4", "--warmup", "3", "--no-extensions"])
     q.put((rank, out.getvalue()))
 
 
@@ -90,5 +91,10 @@ def test_bench_line_over_two_gloo_ranks():
     per_rank = bench.algorithmic_flops(w) / (d["ms_per_step"] * 1e-3) / 1e12
     assert d["n_gpus"] == 2 and d["scaling"] == "weak"
     assert d["value"] == pytest.approx(2 * per_rank)
-    assert d["config"]["parallelism"].startswith("dp2")
     assert "cpu_baseline" not in d  # the oracle baseline runs at one rank only
+    # the benchmark-config rows count both ranks' work too, and carry no oracle figure
+    wm = bench.gi.WORKLOADS["mqa_long"]
+    row = d["rows"]["mqa_long"]
+    assert row["value"] == pytest.approx(2 * bench.algorithmic_flops(wm) / (row["ms_per_step"] * 1e-3) / 1e12,
+                                         rel=1e-3)
+    assert all("cpu_baseline" not in r for r in d["rows"].values())
