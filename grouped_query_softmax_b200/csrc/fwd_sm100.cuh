@@ -28,8 +28,6 @@
 // only, and applies the mask only on tiles that cross its diagonal.
 #pragma once
 
-#include <type_traits>
-
 #include "sm100_ptx.cuh"
 
 namespace gqa {
@@ -46,11 +44,6 @@ constexpr int kFwdSoftmaxRegs = 200;
 static_assert(128 * (kFwdCtlRegs + 2 * kFwdSoftmaxRegs) <= kFwdThreads * kFwdLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between refreshes
-#ifndef GQA_FWD_POLY_EVERY
-#define GQA_FWD_POLY_EVERY 0
-#endif
-// every kPolyEvery-th column pair of an unmasked tile takes the polynomial exp2 (0 = none)
-constexpr int kPolyEvery = GQA_FWD_POLY_EVERY;
 
 constexpr int kUnitPairHeads = 1;
 constexpr int kUnitHeadMajor = 2;
@@ -684,40 +677,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const uint64_t sl2x2 = f2_pack(sl2, sl2);
                 const uint64_t negm2 = f2_pack(neg_m, neg_m);
                 uint64_t lacc[4] = {0ull, 0ull, 0ull, 0ull};
-                // p = 2^(s * scale * log2(e) - m), two columns per packed instruction; on
-                // tiles without masked columns every kPolyEvery-th pair goes through the
-                // FMA-pipe polynomial so the MUFU is not the only exp2 unit.
-                auto exp_pair = [&](uint64_t x, bool poly) -> uint64_t {
-                    if (poly) return exp2_poly_x2(x);
-                    float x0, x1;
-                    f2_unpack(x, x0, x1);
-                    return f2_pack(ex2_approx(x0), ex2_approx(x1));
-                };
-                auto softmax_chunks = [&](auto poly_tag) {
-                    constexpr bool kPoly = decltype(poly_tag)::value;
+                // p = 2^(s * scale * log2(e) - m), two columns per packed instruction
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t pk[16];
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const uint64_t x = f2_fma(
-                                f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
-                                sl2x2, negm2);
-                            const bool use_poly =
-                                kPoly && kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-                            const uint64_t pp = exp_pair(x, use_poly);
-                            lacc[e & 3] = f2_add(lacc[e & 3], pp);
-                            float p0, p1;
-                            f2_unpack(pp, p0, p1);
-                            pk[e] = pack_bf16x2(p0, p1);
-                        }
-                        tmem_st16(tS + c * 16, pk);
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x = f2_fma(
+                            f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sl2x2, negm2);
+                        float x0, x1;
+                        f2_unpack(x, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        lacc[e & 3] = f2_add(lacc[e & 3], f2_pack(p0, p1));
+                        pk[e] = pack_bf16x2(p0, p1);
                     }
-                };
-                if (diag)
-                    softmax_chunks(std::false_type{});
-                else
-                    softmax_chunks(std::true_type{});
+                    tmem_st16(tS + c * 16, pk);
+                }
 
                 {
                     const uint64_t s01 = f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3]));

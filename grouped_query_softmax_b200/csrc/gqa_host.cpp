@@ -14,6 +14,7 @@
 // waits until its output has been copied out.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -85,6 +86,10 @@ cudaError_t copy_rows(void* dst, size_t dst_pitch, const void* src, size_t src_p
     return cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, bytes, planes, kind, s);
 }
 
+// Chunk before whose kernel gqa_attn_fwd_host stops with an error (-1: never); set only
+// through gqa_testing_fwd_host_fail_at, to test the error path.
+std::atomic<int> g_fail_at_chunk{-1};
+
 }  // namespace
 
 extern "C" {
@@ -93,6 +98,12 @@ size_t gqa_attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk,
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tk <= 0 || (D != 64 && D != 128) || Hq % Hkv != 0 || Tq > Tk)
         return 0;
     return plan_host(B, Hq, Hkv, Tq, Tk, D).total;
+}
+
+gqa_status gqa_testing_fwd_host_fail_at(int chunk) {
+    if (chunk < -1 || chunk >= kHostChunks) return GQA_ERR_INVALID_ARGUMENT;
+    g_fail_at_chunk.store(chunk, std::memory_order_relaxed);
+    return GQA_OK;
 }
 
 gqa_status gqa_testing_fwd_host_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int* out_chunks, int* out_row0,
@@ -181,6 +192,10 @@ gqa_status gqa_attn_fwd_host(const void* q, const void* k, const void* v, void* 
             // slot must have been copied out (chunk c - 2)
             if (!ok(cudaStreamWaitEvent(s_main, ev_in[c], 0))) goto done;
             if (c >= 2 && !ok(cudaStreamWaitEvent(s_main, ev_out[c - 2], 0))) goto done;
+            if (c == g_fail_at_chunk.load(std::memory_order_relaxed)) {  // testing hook only
+                result = GQA_ERR_UNSUPPORTED;
+                goto done;
+            }
             st = gqa_attn_fwd_ex(q_slot, k_dev, v_dev, o_slot, lse ? lse_slot : nullptr, B, Hq, Hkv, rows, keys, D,
                                  (long long)Hkv * Tk * D, (long long)Tk * D, (long long)Hkv * Tk * D,
                                  (long long)Tk * D, softmax_scale, window, s_main);
@@ -203,6 +218,13 @@ gqa_status gqa_attn_fwd_host(const void* q, const void* k, const void* v, void* 
         if (!ok(cudaStreamWaitEvent(s_main, ev_out[pl.chunks - 1], 0))) goto done;
     }
 done:
+    if ((result != GQA_OK || e != cudaSuccess) && s_in && s_out) {
+        // an error after some chunks were queued: copies already on the internal streams may
+        // still read the caller's inputs or write its outputs; the call returns only after
+        // they have finished, so the caller may free or reuse its host buffers at once
+        cudaStreamSynchronize(s_in);
+        cudaStreamSynchronize(s_out);
+    }
     // streams and events are released once their work completes
     for (int c = 0; c < kHostChunks; ++c) {
         if (ev_in[c]) cudaEventDestroy(ev_in[c]);

@@ -327,36 +327,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     return d;
 }
 
-// 2^x for a pair, on the FMA pipe instead of the MUFU: Cody-Waite style range
-// reduction x = n + f with n = rint(x) (obtained by adding 1.5 * 2^23, which leaves n
-// in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients were fitted for this library as the minimax relative-error fit on
-// [-1/2, 1/2] (max relative error 7.5e-5 after fp32 evaluation); 2^n is applied by
-// adding n to the exponent field. Inputs are clamped to >= -125 so the result stays
-// a normal number; callers only use it where no input is -inf.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-    // clamp both lanes (no packed max exists), keeping the pair in one 64-bit register
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-    const uint64_t t = f2_add(x, magic);                 // rint(x) in the low mantissa bits
-    const uint64_t f = f2_sub(x, f2_sub(t, magic));      // x - rint(x), in [-1/2, 1/2]
-    uint64_t p = f2_fma(f2_pack(0.05517221987247467f, 0.05517221987247467f), f,
-                        f2_pack(0.24261115491390228f, 0.24261115491390228f));
-    p = f2_fma(p, f, f2_pack(0.6932608485221863f, 0.6932608485221863f));
-    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-    // add n = rint(x) to each lane's exponent field: n << 23 is t's bit pattern << 23
-    uint32_t t0, t1, p0, p1;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
-    p0 += t0 << 23;
-    p1 += t1 << 23;
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(p0), "r"(p1));
-    return r;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     // cvt packs its first source into the upper half

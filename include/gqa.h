@@ -170,9 +170,13 @@ GQA_API gqa_status gqa_attn_decode(const void* q, const void* k_cache, const voi
  * that loads the library, held until the process exits. A call whose partials need
  * more (gqa_attn_decode_workspace_bytes(...) > 16 MiB) returns GQA_ERR_WORKSPACE and
  * launches nothing; num_splits = 1 needs no scratch. Allocates nothing.
- * The first call on each device does a one-time set-up (it looks up the scratch's
- * device address); make that first call before any stream capture. All calls on a
- * device share the scratch and it keeps the last call's contents (nothing needs
+ * The scratch's device address belongs to a CUDA context. The first call in each
+ * context (normally once per device, in the runtime's primary context) does a one-time
+ * set-up: it looks that address up and caches it under the context's ID. Make that
+ * first call before any stream capture. A context created later, for example after
+ * cudaDeviceReset, or a caller's own context, has another ID and gets its own set-up,
+ * so a cached address is never used outside the context it came from. All calls in a
+ * context share the scratch and it keeps the last call's contents (nothing needs
  * clearing: every partial is written before it is read); calls whose kernels can
  * overlap on the GPU race on it.
  */

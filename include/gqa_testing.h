@@ -46,6 +46,15 @@ GQA_API gqa_status gqa_testing_bwd_order(int n_kb, int n_bg, int G, int Tq, int 
 GQA_API gqa_status gqa_testing_fwd_host_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int* out_chunks,
                                              int* out_row0, int* out_rows, int* out_keys);
 
+/*
+ * Makes every later gqa_attn_fwd_host call stop with GQA_ERR_UNSUPPORTED just before the
+ * kernel of chunk `chunk` (0 <= chunk < 8), after the earlier chunks' kernels and copies
+ * were queued, so that tests can check the error path: such a call returns only once the
+ * copies it queued have finished. -1 switches the hook off (the default). Process-wide;
+ * touches no GPU. Returns GQA_ERR_INVALID_ARGUMENT for other values.
+ */
+GQA_API gqa_status gqa_testing_fwd_host_fail_at(int chunk);
+
 #ifdef __cplusplus
 }
 #endif

@@ -147,3 +147,39 @@ def test_peaked_softmax_stability(gqa):
     q, k, v = rand_qkv(2, 4, 4, 256, 1024, 128, seed=10, q_pow2=2)
     got = from_dev(run_fwd(gqa, q, k, v))
     assert_parity(got, oracle.attention(q, k, v), "peaked")
+
+
+def test_boundary_entry_points_by_name(gqa):
+    """gqa_attn_fwd and gqa_attn_decode themselves (not their extended siblings), called by
+    name through the C ABI with raw device pointers, against the fp64 oracle."""
+    torch = torch_mod()
+    stream = torch.cuda.current_stream().cuda_stream
+    B, Hq, Hkv, Tq, Tk, D = 2, 8, 2, 300, 1111, 128            # suffix offset 811, ragged tiles
+    q, k, v = rand_qkv(B, Hq, Hkv, Tq, Tk, D, seed=41)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    od = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, Hq, Tq), float("nan"), dtype=torch.float32, device=qd.device)
+    st = gqa.gqa_attn_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), lse.data_ptr(),
+                          B, Hq, Hkv, Tq, Tk, D, kd.stride(0), kd.stride(1), vd.stride(0), vd.stride(1), 0.0, stream)
+    assert st == gqa.GQA_OK, gqa.gqa_status_string(st)
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_device_error() == gqa.GQA_OK
+    ref, ref_lse = oracle.attention(q, k, v, with_lse=True)
+    assert_parity(from_dev(od), ref, "gqa_attn_fwd by name")
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 1e-3
+
+    Bd, Tkd = 4, 5000                                          # decode over several splits
+    qd1, kd1, vd1 = rand_qkv(Bd, Hq, Hkv, 1, Tkd, D, seed=42)
+    splits = gqa.gqa_attn_decode_num_splits(Bd, Hq, Hkv, Tkd, D, 0)
+    assert splits > 1
+    need = gqa.gqa_attn_decode_workspace_bytes(Bd, Hq, Hkv, Tkd, D, 0)
+    ws = torch.empty(need, dtype=torch.uint8, device=qd.device)
+    qq, kk, vv = to_dev(qd1), to_dev(kd1), to_dev(vd1)
+    oo = torch.full_like(qq, float("nan"))
+    st = gqa.gqa_attn_decode(qq.data_ptr(), kk.data_ptr(), vv.data_ptr(), oo.data_ptr(), Bd, Hq, Hkv, Tkd, D,
+                             kk.stride(0), kk.stride(1), vv.stride(0), vv.stride(1), 0.0, 0, ws.data_ptr(), need,
+                             stream)
+    assert st == gqa.GQA_OK, gqa.gqa_status_string(st)
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_device_error() == gqa.GQA_OK
+    assert_parity(from_dev(oo), oracle.attention(qd1, kd1, vd1), "gqa_attn_decode by name")

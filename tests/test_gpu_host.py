@@ -67,3 +67,28 @@ def test_host_call_full_size_gqa_prefill(gqa):
     o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v))
     o_host = gqa.attn_fwd_host(host_bf16(q), host_bf16(k), host_bf16(v))
     np.testing.assert_array_equal(u16(o_host), u16(o_dev))
+
+
+def test_host_call_error_returns_after_its_queued_copies(gqa):
+    """An error after some chunks were queued (forced by the testing hook before chunk 2's
+    kernel) returns only once the copies already queued have finished: the output rows of
+    chunks 0 and 1 are in host memory when the call returns, with no synchronisation."""
+    import ctypes
+    lib = ctypes.CDLL(gqa.library_path())
+    B, Hq, Hkv, Tq, Tk, D = 2, 8, 2, 2048, 2048, 128          # 8 chunks of 256 rows
+    w = gi.Workload("host error path", B, Hq, Hkv, Tq, Tk, D, seed=139)
+    q, k, v = w.make()
+    o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v))
+    torch = torch_mod()
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16).pin_memory()
+    assert lib.gqa_testing_fwd_host_fail_at(2) == 0
+    try:
+        with pytest.raises(gqa.GqaError):
+            gqa.attn_fwd_host(host_bf16(q), host_bf16(k), host_bf16(v), out=out, synchronize=False)
+        got = out.view(torch.int16).numpy().view(np.uint16)    # read at once: no synchronisation
+        np.testing.assert_array_equal(got[:, :, :512], u16(o_dev)[:, :, :512])
+    finally:
+        assert lib.gqa_testing_fwd_host_fail_at(-1) == 0
+    assert lib.gqa_testing_fwd_host_fail_at(8) == gqa.GQA_ERR_INVALID_ARGUMENT
+    o_host = gqa.attn_fwd_host(host_bf16(q), host_bf16(k), host_bf16(v))
+    np.testing.assert_array_equal(u16(o_host), u16(o_dev))
