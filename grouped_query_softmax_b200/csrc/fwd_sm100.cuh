@@ -655,22 +655,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                          max3f(max3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
                 const float m_new = fmaxf(m, tmax * sl2);
                 const bool refresh = m_new > m + kRescaleThreshold;
-                const float alpha = refresh ? ex2_approx(m - m_new) : 1.f;
-                l *= alpha;
-                m = refresh ? m_new : m;
-                if (j > me.j_begin && __any_sync(0xffffffffu, refresh)) {
-                    // O_s has absorbed all earlier P V products (their completion is
-                    // ordered before S_j's commit); rescale this row in place.
+                // warp-uniform branch, rarely taken after a unit's first tile: the MUFU op for
+                // alpha stays off the common path (it would queue behind the exponentials)
+                if (__any_sync(0xffffffffu, refresh)) {
+                    const float alpha = refresh ? ex2_approx(m - m_new) : 1.f;
+                    l *= alpha;
+                    m = refresh ? m_new : m;
+                    if (j > me.j_begin) {
+                        // O_s has absorbed all earlier P V products (their completion is
+                        // ordered before S_j's commit); rescale this row in place.
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t orr[32];
-                        tmem_ld32(tO + c * 32, orr);
-                        tc_wait_ld();
-                        reg_fence32(orr);
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t orr[32];
+                            tmem_ld32(tO + c * 32, orr);
+                            tc_wait_ld();
+                            reg_fence32(orr);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32(tO + c * 32, orr);
+                            for (int e = 0; e < 32; ++e)
+                                orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                            tmem_st32(tO + c * 32, orr);
+                        }
                     }
                 }
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
