@@ -17,7 +17,8 @@ import ctypes
 import os
 
 __all__ = [
-    "GqaError", "gqa_attn_fwd", "gqa_attn_fwd_ex", "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
+    "GqaError", "gqa_attn_fwd", "gqa_attn_fwd_ex", "gqa_attn_fwd_split", "gqa_attn_fwd_split_workspace_bytes",
+    "gqa_attn_decode", "gqa_attn_decode_workspace_bytes",
     "gqa_attn_decode_num_splits", "gqa_attn_decode_static", "gqa_attn_decode_ex",
     "gqa_attn_decode_ex_workspace_bytes", "gqa_attn_decode_ex_num_splits", "gqa_status_string", "gqa_get_device_error",
     "gqa_selftest_bounded_wait", "attn_fwd", "attn_decode", "library_path",
@@ -54,6 +55,11 @@ _lib.gqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _
 _lib.gqa_attn_fwd_ex.restype = _i32
 _lib.gqa_attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                  _ll, _ll, _ll, _ll, _f32, _i32, _vp]
+_lib.gqa_attn_fwd_split_workspace_bytes.restype = _sz
+_lib.gqa_attn_fwd_split_workspace_bytes.argtypes = [_i32] * 7
+_lib.gqa_attn_fwd_split.restype = _i32
+_lib.gqa_attn_fwd_split.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                    _ll, _ll, _ll, _ll, _f32, _i32, _vp, _sz, _vp]
 _lib.gqa_attn_fwd_host_workspace_bytes.restype = _sz
 _lib.gqa_attn_fwd_host_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32]
 _lib.gqa_attn_fwd_host.restype = _i32
@@ -131,6 +137,19 @@ def gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_
     """C ``gqa_attn_fwd_ex``: ``gqa_attn_fwd`` with a sliding window (0 = causal only)."""
     return _lib.gqa_attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
                                 float(softmax_scale), int(window), stream)
+
+
+def gqa_attn_fwd_split_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window=0) -> int:
+    """C ``gqa_attn_fwd_split_workspace_bytes`` (0: the launch does not split)."""
+    return _lib.gqa_attn_fwd_split_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window)
+
+
+def gqa_attn_fwd_split(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                       softmax_scale=0.0, window=0, workspace=None, workspace_bytes=0, stream=None) -> int:
+    """C ``gqa_attn_fwd_split``: ``gqa_attn_fwd_ex`` that may split the keys of the last wave's
+    units over several CTAs (partials merged by log-sum-exp in a workspace). Returns the status."""
+    return _lib.gqa_attn_fwd_split(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh,
+                                   float(softmax_scale), window, workspace, workspace_bytes, stream)
 
 
 def gqa_attn_fwd_host_workspace_bytes(B, Hq, Hkv, Tq, Tk, D) -> int:
@@ -290,12 +309,19 @@ def _plane_strides(t, name):
     return t.stride(0), t.stride(1)
 
 
-def attn_fwd(q, k, v, *, Tk=None, scale=None, window=0, return_lse=False, out=None, stream=None):
+def attn_fwd(q, k, v, *, Tk=None, scale=None, window=0, return_lse=False, out=None, stream=None, split=True,
+             workspace=None):
     """o = causal GQA attention of q [B,Hq,Tq,D] over k, v [B,Hkv,T_cap,D] (first Tk rows).
 
     Query row i sits at position Tk - Tq + i; ``window`` > 0 limits it to its
     ``window`` most recent positions. Returns o (bf16, [B,Hq,Tq,D]) and, if
     ``return_lse``, the fp32 natural-log log-sum-exp [B,Hq,Tq].
+
+    With ``split`` (the default) the call goes through gqa_attn_fwd_split, which may
+    split the keys of the last wave's units over several CTAs (the results then agree with
+    ``split=False``, gqa_attn_fwd_ex, within rounding rather than bit for bit);
+    ``workspace`` is then a uint8 CUDA tensor of at least
+    gqa_attn_fwd_split_workspace_bytes(...) bytes, allocated here when omitted.
     """
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -314,12 +340,23 @@ def attn_fwd(q, k, v, *, Tk=None, scale=None, window=0, return_lse=False, out=No
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
-    st = gqa_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                         lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Tq, Tk, D,
-                         k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), int(window),
-                         _stream_handle(stream))
+    lse_ptr = lse.data_ptr() if lse is not None else None
+    if not split:
+        st = gqa_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Tq, Tk,
+                             D, k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), int(window), _stream_handle(stream))
+        if st != GQA_OK:
+            raise GqaError(st, "gqa_attn_fwd_ex")
+        return (out, lse) if return_lse else out
+    need = gqa_attn_fwd_split_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, int(window))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if (need and workspace is not None) else 0
+    st = gqa_attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Tq, Tk, D,
+                            k_sb, k_sh, v_sb, v_sh, float(scale or 0.0), int(window), ws_ptr, ws_bytes,
+                            _stream_handle(stream))
     if st != GQA_OK:
-        raise GqaError(st, "gqa_attn_fwd_ex")
+        raise GqaError(st, "gqa_attn_fwd_split")
     return (out, lse) if return_lse else out
 
 

@@ -63,6 +63,12 @@ struct FwdParams {
     float* lse;  // nullable
     uint32_t* err;
     unsigned long long timeout_ns;
+    // split launches: units from split_whole on are parts, split_k per unit, each covering
+    // a k-th of that unit's key tiles; they write fp32 O / l rows to part and their
+    // log2-domain log-sum-exp to part_lse (split_k <= 1: no parts)
+    int split_whole, split_k;
+    float* part;
+    float* part_lse;
 };
 
 // Sequences of different lengths (the kVarlen instantiation only). A kernel parameter
@@ -182,6 +188,32 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
     fwd_fill_subtile(st[1], p.Tq, off, p.window);
 }
 
+// Part index of unit u of a split launch (-1 for a whole unit) and the unit it is a part of.
+__device__ __forceinline__ int fwd_split_part(const FwdParams& p, int u, int& base) {
+    if (p.split_k <= 1 || u < p.split_whole) {
+        base = u;
+        return -1;
+    }
+    const int v = u - p.split_whole;
+    const int su = v / p.split_k;
+    base = p.split_whole + su;
+    return v - su * p.split_k;
+}
+
+// Part `part` of `k` of a unit covers key tiles [n * part / k, n * (part + 1) / k) of its
+// n = longest sub-tile's tiles; each sub-tile keeps the tiles of its own range inside it.
+__device__ __forceinline__ void fwd_clamp_part(SubTile (&st)[2], int part, int k) {
+    const int n_max = max(st[0].n_kv, st[1].n_kv);
+    const int j0 = n_max * part / k, j1 = n_max * (part + 1) / k;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        if (st[s].n_kv == 0) continue;
+        st[s].j_begin = max(st[s].j_begin, j0);
+        st[s].n_kv = min(st[s].n_kv, j1);
+        if (st[s].j_begin >= st[s].n_kv) st[s].n_kv = 0;
+    }
+}
+
 // One sequence side: batch index, first row and length.
 __device__ __forceinline__ void fwd_seq_side(const int* cu, const int* len, int rows, int s, int& b,
                                              int& r, int& l) {
@@ -236,8 +268,10 @@ __device__ __forceinline__ void fwd_unit(const FwdParams& p, const FwdVarlenPara
     if constexpr (kVarlen) {
         fwd_varlen_unit(p, vp, __ldg(vp.unit_list + u), geo, g, st);
     } else {
-        int b;
-        fwd_decode_unit(p, u, b, g, st);
+        int b, base;
+        const int part = fwd_split_part(p, u, base);
+        fwd_decode_unit(p, base, b, g, st);
+        if (part >= 0) fwd_clamp_part(st, part, p.split_k);
         geo.b_q = geo.b_k = b;
         geo.r_q = geo.r_k = 0;
         geo.len_q = p.Tq;
@@ -713,6 +747,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 break;
             oph ^= 1u;
             tc_fence_after_sync();
+            int part = -1, base_u = u;
+            if constexpr (!kVarlen) part = fwd_split_part(p, u, base_u);
+            if (part >= 0) {
+                // a part of a split unit: fp32 O / l and the log2-domain log-sum-exp of this
+                // row over the part's keys (a row that saw none writes zeros and -inf); the
+                // combine kernel merges the parts
+                const size_t prow = ((size_t)(u - p.split_whole) * 2 + s) * kFwdRows + r;
+                const bool any = l > 0.f;
+                const float inv_l = any ? 1.f / l : 0.f;
+                float4* dst = reinterpret_cast<float4*>(p.part + prow * D);
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + c * 32, orr);
+                    tc_wait_ld();
+                    reg_fence32(orr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[c * 8 + e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
+                                                     __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
+                }
+                tc_fence_before_sync();
+                mbar_arrive(smem_u32(&ctl->o_empty[s]));
+                p.part_lse[prow] = any ? m + __log2f(l) : -INFINITY;
+                continue;
+            }
             const int row = me.row0 + r;
             const bool row_ok = row < geo.len_q;
             const float inv_l = 1.f / l;
@@ -758,6 +818,70 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
 }
 
+
+// ---------------------------------------------------------------- split-launch merge
+// Row r of sub-tile s of split unit su has split_k partial rows: fp32 O / l over a k-th of
+// its keys and the log2-domain log-sum-exp of those keys. With M the largest of them and
+// w_q = 2^(lse_q - M), the row is O = sum_q w_q O_q / sum_q w_q with log-sum-exp
+// M + log2(sum_q w_q): the same merge as the split-KV decode partials, in fixed part order.
+// One warp per row; each lane merges D / 32 consecutive columns.
+constexpr int kCombineWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    gqa_fwd_split_combine_kernel(const FwdParams p, long long n_rows) {
+    const long long w = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    if (w >= n_rows) return;  // n_rows = split units x 2 sub-tiles x 128 rows
+    const int lane = threadIdx.x & 31;
+    const int su = (int)(w >> 8);
+    const int s = (int)(w >> 7) & 1;
+    const int r = (int)w & (kFwdRows - 1);
+    int b, g;
+    SubTile st[2];
+    fwd_decode_unit(p, p.split_whole + su, b, g, st);
+    const int row = st[s].row0 + r;
+    if (st[s].n_kv == 0 || row >= p.Tq) return;  // no such sub-tile, or a row past T_q
+    const int k = p.split_k;
+    const size_t base = ((size_t)su * k * 2 + s) * kFwdRows + r;  // part q: base + q * 2 * 128
+    const size_t stride = 2 * kFwdRows;
+    float M = -INFINITY;
+    for (int q = 0; q < k; ++q) M = fmaxf(M, p.part_lse[base + q * stride]);
+    constexpr int kPer = D / 32;
+    float acc[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+    float wsum = 0.f;
+    for (int q = 0; q < k; ++q) {
+        const float lq = p.part_lse[base + q * stride];
+        if (lq == -INFINITY) continue;  // the part held no key of this row
+        const float wq = ex2_approx(lq - M);
+        wsum += wq;
+        const float* src = p.part + (base + q * stride) * D + lane * kPer;
+        if constexpr (kPer == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            acc[0] += wq * v.x;
+            acc[1] += wq * v.y;
+            acc[2] += wq * v.z;
+            acc[3] += wq * v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            acc[0] += wq * v.x;
+            acc[1] += wq * v.y;
+        }
+    }
+    const float inv = 1.f / wsum;  // > 0: every row sees at least one key in some part
+    __nv_bfloat16* out = p.o + (((size_t)b * p.Hq + st[s].head) * (size_t)p.Tq + row) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+        uint2 pk;
+        pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(out) = pk;
+    } else {
+        *reinterpret_cast<uint32_t*>(out) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+    if (p.lse != nullptr && lane == 0)
+        p.lse[((size_t)b * p.Hq + st[s].head) * (size_t)p.Tq + row] = (M + __log2f(wsum)) * 0.69314718055994530942f;
+}
 
 // ---------------------------------------------------------------- variable-length plan
 // One CTA. Checks every sequence's bounds against the tensors, then lists the units

@@ -166,6 +166,54 @@ gqa_status check_decode(int B, int Hq, int Hkv, int Tq, int Tk, int D, int windo
     return GQA_OK;
 }
 
+gqa_status current_sms(int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return GQA_ERR_CUDA;
+    return GQA_OK;
+}
+
+// gqa_attn_fwd_ex, and with allow_split gqa_attn_fwd_split (a workspace for the parts of a
+// split launch, when the plan splits).
+gqa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int Tq, int Tk, int D, long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                    float softmax_scale, int window, void* workspace, size_t workspace_bytes, bool allow_split,
+                    void* stream) {
+    gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
+    if (st != GQA_OK) return st;
+    if (window < 0) return GQA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GQA_ERR_INVALID_ARGUMENT;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+
+    gqa::FwdLaunch a{};
+    a.window = window >= Tk ? 0 : window;  // a window covering every key is plain causal
+    a.split_k = 1;
+    if (allow_split) {
+        int sms = 0;
+        if ((st = current_sms(&sms)) != GQA_OK) return st;
+        const gqa::FwdSplitPlan sp = gqa::fwd_split_plan(B, Hq, Hkv, Tq, Tk, a.window, sms);
+        const size_t need = gqa::fwd_split_workspace_bytes(sp, D);
+        if (need > 0) {
+            if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+                return GQA_ERR_WORKSPACE;
+            a.split_k = sp.k;
+            a.part = static_cast<float*>(workspace);
+        }
+    }
+    const long long q_sh = (long long)Tq * D;
+    if ((st = make_map(&a.tm_q, q, B, Hq, Tq, D, q_sh * Hq, q_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    a.o = o;
+    a.lse = lse;
+    return gqa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -193,26 +241,24 @@ gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
                            int Hq, int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh,
                            long long v_sb, long long v_sh, float softmax_scale, int window,
                            void* stream) {
-    gqa_status st = check_common(B, Hq, Hkv, Tq, Tk, D);
-    if (st != GQA_OK) return st;
-    if (window < 0) return GQA_ERR_INVALID_ARGUMENT;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GQA_ERR_INVALID_ARGUMENT;
-    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_INVALID_ARGUMENT;
-    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return GQA_ERR_INVALID_ARGUMENT;
-    if ((st = check_kv_strides(B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
-    if ((st = check_kv_strides(B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh, softmax_scale, window,
+                    nullptr, 0, false, stream);
+}
 
-    gqa::FwdLaunch a{};
-    const long long q_sh = (long long)Tq * D;
-    if ((st = make_map(&a.tm_q, q, B, Hq, Tq, D, q_sh * Hq, q_sh)) != GQA_OK) return st;
-    if ((st = make_map(&a.tm_k, k, B, Hkv, Tk, D, k_sb, k_sh)) != GQA_OK) return st;
-    if ((st = make_map(&a.tm_v, v, B, Hkv, Tk, D, v_sb, v_sh)) != GQA_OK) return st;
-    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Tq = Tq; a.Tk = Tk; a.D = D;
-    a.window = window >= Tk ? 0 : window;  // a window covering every key is plain causal
-    a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
-    a.o = o;
-    a.lse = lse;
-    return gqa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+size_t gqa_attn_fwd_split_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window) {
+    if (check_common(B, Hq, Hkv, Tq, Tk, D) != GQA_OK || window < 0) return 0;
+    int sms = 0;
+    if (current_sms(&sms) != GQA_OK) return 0;
+    return gqa::fwd_split_workspace_bytes(
+        gqa::fwd_split_plan(B, Hq, Hkv, Tq, Tk, window >= Tk ? 0 : window, sms), D);
+}
+
+gqa_status gqa_attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int Tq, int Tk, int D, long long k_sb, long long k_sh, long long v_sb,
+                              long long v_sh, float softmax_scale, int window, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Tq, Tk, D, k_sb, k_sh, v_sb, v_sh, softmax_scale, window,
+                    workspace, workspace_bytes, true, stream);
 }
 
 int gqa_attn_decode_ex_num_splits(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window,
@@ -498,6 +544,18 @@ gqa_status gqa_get_device_error(void* stream) {
     if (gqa::read_and_clear_device_error(&v) != cudaSuccess) return GQA_ERR_CUDA;
     if (v & gqa::kErrBitWaitTimeout) return GQA_ERR_TIMEOUT;
     if (v & gqa::kErrBitBadSeqlens) return GQA_ERR_INVALID_ARGUMENT;
+    return GQA_OK;
+}
+
+gqa_status gqa_testing_fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window, int sms,
+                                      int* out_k, long long* out_whole, long long* out_split, long long* out_units) {
+    if (!out_k || !out_whole || !out_split || !out_units || sms < 1 || window < 0) return GQA_ERR_INVALID_ARGUMENT;
+    if (check_common(B, Hq, Hkv, Tq, Tk, D) != GQA_OK) return GQA_ERR_INVALID_ARGUMENT;
+    const gqa::FwdSplitPlan sp = gqa::fwd_split_plan(B, Hq, Hkv, Tq, Tk, window >= Tk ? 0 : window, sms);
+    *out_k = sp.k;
+    *out_whole = sp.whole;
+    *out_split = sp.split;
+    *out_units = gqa::fwd_units(B, Hq, Hkv, Tq);
     return GQA_OK;
 }
 

@@ -15,7 +15,74 @@ struct FwdLaunch {
     float scale;
     void* o;
     float* lse;
+    // split launch (fwd_split_plan): the last units' key tiles in split_k parts, whose
+    // fp32 partials go to `part` and are merged by a second kernel; split_k <= 1: none
+    int split_k;
+    float* part;
 };
+
+// Work units of a dense forward launch: pairs of 128-row sub-tiles (heads a, a+1 of one
+// group when the group size is even, else rows r and r + 128 of one head).
+inline long long fwd_units(int B, int Hq, int Hkv, int Tq) {
+    const int G = Hq / Hkv;
+    const int n_qt = (Tq + 127) / 128;
+    return G % 2 == 0 ? (long long)B * Hkv * (G / 2) * n_qt : (long long)B * Hq * ((n_qt + 1) / 2);
+}
+
+// Split plan of a dense forward launch on `sms` persistent CTAs. Only plain causal suffix
+// launches whose cached prefix is at least as long as the suffix qualify: their units all
+// have about the same number of key tiles n, so a last wave of r = units mod sms units
+// leaves sms - r CTAs idle for a whole unit. Those r units are cut into k parts of about
+// n / k tiles (at least 2), which the persistent CTAs take after the whole units; k (at
+// most 8) minimises the estimated makespan (whole waves x n + part waves x (n / k + c),
+// c = kFwdSplitPartCost tiles standing for a part's fixed cost: its Q load, pipeline fill,
+// fp32 partial rows and share of the merge) and is used only if that estimate beats no
+// split by 10 %. Partial rows: split units x k x 2 sub-tiles x 128 rows.
+struct FwdSplitPlan {
+    int k = 1;           // parts per split unit (1: no split)
+    long long whole = 0; // units run whole (they come first in the unit list)
+    long long split = 0; // units cut into k parts
+    long long rows = 0;  // partial rows written to the workspace
+};
+constexpr int kFwdSplitMaxParts = 8;
+// Fixed cost of a part, in key tiles: the MHA suffix workload (256 units of 64 tiles on 148
+// SMs) measured 2.5 % slower split in 4 than whole, which puts it near 5 tiles.
+constexpr double kFwdSplitPartCost = 5.0;
+inline FwdSplitPlan fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int window, int sms) {
+    FwdSplitPlan sp;
+    const long long units = fwd_units(B, Hq, Hkv, Tq);
+    sp.whole = units;
+    if (window > 0 || Tk - Tq < Tq || sms <= 0 || units <= 0) return sp;
+    const long long n = (Tk - 1) / 128 + 1;  // key tiles of a unit's last row
+    const long long full = units / sms, r = units % sms;
+    if (r == 0) return sp;
+    const double base = (double)(full + 1) * n;
+    double best = base;
+    int best_k = 1;
+    for (int k = 2; k <= kFwdSplitMaxParts && n / k >= 2; ++k) {
+        const long long part_waves = (r * k + sms - 1) / sms;
+        const double cost = (double)full * n + (double)part_waves * ((double)n / k + kFwdSplitPartCost);
+        if (cost < best) {
+            best = cost;
+            best_k = k;
+        }
+    }
+    if (best_k == 1 || best > 0.9 * base) return sp;
+    sp.k = best_k;
+    sp.whole = units - r;
+    sp.split = r;
+    sp.rows = r * best_k * 2 * 128;
+    return sp;
+}
+// Workspace of a split launch: fp32 partial O rows [rows, D], then their log2-domain
+// log-sum-exp [rows] (each 256-byte aligned).
+inline size_t fwd_split_lse_offset(long long rows, int D) {
+    return ((size_t)rows * D * sizeof(float) + 255) & ~(size_t)255;
+}
+inline size_t fwd_split_workspace_bytes(const FwdSplitPlan& sp, int D) {
+    if (sp.k <= 1) return 0;
+    return fwd_split_lse_offset(sp.rows, D) + (size_t)sp.rows * sizeof(float);
+}
 
 // Sequences of different lengths (gqa_attn_fwd_varlen). Exactly one of cu_* / len_*
 // describes each side (both null: every sequence owns all rows of its batch).

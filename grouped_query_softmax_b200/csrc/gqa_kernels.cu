@@ -53,13 +53,25 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     p.err = device_error_ptr();
     p.timeout_ns = kWaitTimeoutNs;
     if (!p.err) return cudaErrorUnknown;
-    if (units <= 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    p.units = (int)units;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    FwdSplitPlan sp;
+    p.split_k = 1;
+    if (a.split_k > 1) {
+        // the caller sized its workspace with the same plan on the same device
+        sp = fwd_split_plan(a.B, a.Hq, a.Hkv, a.Tq, a.Tk, a.window, sms);
+        if (sp.k != a.split_k || !a.part || units != sp.whole + sp.split) return cudaErrorInvalidValue;
+        p.split_whole = (int)sp.whole;
+        p.split_k = sp.k;
+        p.part = a.part;
+        p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(a.part) + fwd_split_lse_offset(sp.rows, D));
+        units = sp.whole + sp.split * sp.k;
+    }
+    if (units <= 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.units = (int)units;
     const int smem = FwdSmem<D>::kBytes;
     e = cudaFuncSetAttribute(gqa_fwd_sm100_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -73,6 +85,12 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     const unsigned grid = (unsigned)std::min<long long>(units, sms > 0 ? sms : 1);
     gqa_fwd_sm100_kernel<D, false><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p,
                                                                          FwdVarlenParams{});
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.split_k <= 1) return e;
+    // merge the parts of the split units (stream order makes their partials visible)
+    const long long rows = sp.split * 2 * kFwdRows;
+    const long long blocks = (rows + kCombineWarps - 1) / kCombineWarps;
+    gqa_fwd_split_combine_kernel<D><<<(unsigned)blocks, kCombineWarps * 32, 0, stream>>>(p, rows);
     return cudaGetLastError();
 }
 

@@ -95,6 +95,38 @@ GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, 
                                    float softmax_scale, int window, void* stream);
 
 /*
+ * gqa_attn_fwd_ex with a caller workspace that lets the library split the keys of some work
+ * units over several CTAs. The operation is the same o_a definition ("注意力家族", section
+ * 统一记号, with the causal suffix mask of its section 最小语义实现); only the order in which
+ * the keys of a row are summed changes, so results agree with gqa_attn_fwd_ex within rounding
+ * (not bit for bit).
+ *
+ * Which launches split: plain causal suffix calls (window = 0) whose cached prefix is at
+ * least as long as the suffix (T_k - T_q >= T_q). Their work units (pairs of 128-row query
+ * tiles) all need about the same number of key tiles, so when their count is not a multiple
+ * of the number of SMs the last wave of the persistent kernel leaves SMs idle. The units of
+ * that last wave are then cut into 2 to 8 parts along the keys; each part writes its rows'
+ * fp32 partial output and log-sum-exp to the workspace, and a second kernel merges them by
+ * log-sum-exp (the same merge as decode's split-KV partials). The tile splitting that
+ * "A Visual Guide to Attention", section "Sources and execution", describes for one row is
+ * here spread over CTAs.
+ *
+ *   workspace, workspace_bytes  device memory of at least
+ *            gqa_attn_fwd_split_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window) bytes (same
+ *            arguments, same current device), 256-byte aligned, caller-owned. Its contents on
+ *            entry are ignored; it must not be shared by calls that can overlap on the GPU.
+ *            When that size is 0 the launch does not split and workspace may be NULL.
+ *            A missing, misaligned or smaller workspace is GQA_ERR_WORKSPACE.
+ * Other arguments and errors as gqa_attn_fwd_ex.
+ */
+GQA_API size_t gqa_attn_fwd_split_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window);
+GQA_API gqa_status gqa_attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse,
+                                      int B, int Hq, int Hkv, int Tq, int Tk, int D,
+                                      long long k_sb, long long k_sh, long long v_sb, long long v_sh,
+                                      float softmax_scale, int window, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/*
  * gqa_attn_fwd_ex for operands in HOST memory, for callers whose tensors are not yet on the
  * device. The pages define the operation only; moving operands is a library convenience.
  *

@@ -46,7 +46,7 @@ def test_host_call_equals_device_call_bitwise(gqa, case):
     B, Hq, Hkv, Tq, Tk, D, win = case
     w = gi.Workload("host test", B, Hq, Hkv, Tq, Tk, D, seed=131)
     q, k, v = w.make()
-    o_dev, lse_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v), window=win, return_lse=True)
+    o_dev, lse_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v), window=win, return_lse=True, split=False)
     o_host, lse_host = gqa.attn_fwd_host(host_bf16(q), host_bf16(k), host_bf16(v), window=win, return_lse=True)
     assert gqa.gqa_get_device_error() == gqa.GQA_OK
     np.testing.assert_array_equal(u16(o_host), u16(o_dev))
@@ -64,7 +64,7 @@ def test_host_call_matches_oracle_with_pageable_memory(gqa):
 def test_host_call_full_size_gqa_prefill(gqa):
     w = gi.WORKLOADS["gqa_prefill"]
     q, k, v = w.make()
-    o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v))
+    o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v), split=False)
     o_host = gqa.attn_fwd_host(host_bf16(q), host_bf16(k), host_bf16(v))
     np.testing.assert_array_equal(u16(o_host), u16(o_dev))
 
@@ -78,7 +78,7 @@ def test_host_call_error_returns_after_its_queued_copies(gqa):
     B, Hq, Hkv, Tq, Tk, D = 2, 8, 2, 2048, 2048, 128          # 8 chunks of 256 rows
     w = gi.Workload("host error path", B, Hq, Hkv, Tq, Tk, D, seed=139)
     q, k, v = w.make()
-    o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v))
+    o_dev = gqa.attn_fwd(to_dev(q), to_dev(k), to_dev(v), split=False)
     torch = torch_mod()
     out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16).pin_memory()
     assert lib.gqa_testing_fwd_host_fail_at(2) == 0
