@@ -45,6 +45,10 @@ static_assert(128 * (kFwdCtlRegs + 2 * kFwdSoftmaxRegs) <= kFwdThreads * kFwdLau
               "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between refreshes
 
+// Readers of a published unit in a dynamic-fetch launch: the MMA thread, the eight softmax
+// warps and the ragged-tile cleaner warp.
+constexpr int kUnitReaders = 10;
+
 constexpr int kUnitPairHeads = 1;
 constexpr int kUnitHeadMajor = 2;
 
@@ -80,8 +84,12 @@ struct FwdVarlenParams {
     const int* len_k; // padded keys; a null length array means every sequence has all rows
     int rows_q, rows_k;  // row extent of the q/o and k/v tensors
     int n_lvl, n_h;      // candidate unit c = (s * n_lvl + level) * n_h + head slot
-    const int* unit_list;   // present units, longest first (written by the plan kernel)
+    const int* unit_list;   // present units (written by the plan kernel)
     const int* unit_count;  // their number
+    // dynamic != 0: the list is sequence-major and the persistent CTAs take its entries in
+    // order through the counter *fetch (zeroed by the plan kernel) instead of a fixed stride
+    int* fetch;
+    int dynamic;
     long long o_sb, o_sh, o_st;  // element strides of o (batch, head, row); d is contiguous
     // paged keys (table non-null): key t of sequence s is row t % page_size of pool page
     // table[s * max_pages + t / page_size]; the k/v tensor maps cover the pool
@@ -115,6 +123,9 @@ struct FwdSmem {
         uint64_t o_full[2];
         uint64_t o_empty[2];
         uint64_t drain;
+        uint64_t unit_full[4];   // dynamic unit fetch: the producer publishes the CTA's k-th unit
+        uint64_t unit_empty[4];  // in slot k % 4; its readers release the slot
+        int unit_ring[4];
         uint32_t tmem_base;
         uint32_t abort;
     };
@@ -285,6 +296,40 @@ __device__ __forceinline__ int snake_unit(int k, int i, int n) {
     return k * n + ((k & 1) ? (n - 1 - i) : i);
 }
 
+// The k-th unit of a persistent CTA as a list index, -1 when the CTA has no more, -2 when a
+// bounded wait gave up. Static launches stride over the list (snake_unit); dynamic ones take
+// the next free entry with an atomic counter, and the producer publishes it in a 4-slot ring
+// that every other role reads (fwd_read_unit) and releases.
+template <class Ctl>
+__device__ __forceinline__ int fwd_publish_unit(Ctl* ctl, int* fetch, int units, int k, volatile uint32_t* abort_flag,
+                                                uint32_t* err, unsigned long long timeout_ns) {
+    const int slot = k & 3;
+    if (k >= 4 && !mbar_wait_bounded(smem_u32(&ctl->unit_empty[slot]), ((k >> 2) - 1) & 1u, abort_flag, err,
+                                     timeout_ns))
+        return -2;
+    const int idx = atomicAdd(fetch, 1);
+    const int u = idx < units ? idx : -1;
+    reinterpret_cast<volatile int*>(ctl->unit_ring)[slot] = u;
+    mbar_arrive(smem_u32(&ctl->unit_full[slot]));  // release: the ring entry is visible to its readers
+    return u;
+}
+// Read the k-th published unit (every lane of the calling warp reads it); lane 0 releases the
+// slot for the warp (one_thread: the caller is a single thread and releases it itself).
+template <class Ctl>
+__device__ __forceinline__ int fwd_read_unit(Ctl* ctl, int k, bool one_thread, volatile uint32_t* abort_flag,
+                                             uint32_t* err, unsigned long long timeout_ns) {
+    const int slot = k & 3;
+    if (!mbar_wait_bounded(smem_u32(&ctl->unit_full[slot]), (k >> 2) & 1u, abort_flag, err, timeout_ns)) return -2;
+    const int u = reinterpret_cast<volatile int*>(ctl->unit_ring)[slot];
+    if (one_thread) {
+        mbar_arrive(smem_u32(&ctl->unit_empty[slot]));
+    } else {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ctl->unit_empty[slot]));
+    }
+    return u;
+}
+
 template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     gqa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -315,6 +360,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int ncta = gridDim.x;
     // variable-length launches read the unit count the plan kernel wrote
     const int units = kVarlen ? *reinterpret_cast<const volatile int*>(vp.unit_count) : p.units;
+    const bool dyn = kVarlen && vp.dynamic != 0;
+    // static launches: the k-th unit of this CTA on the boustrophedon walk (-1: none left)
+    auto static_unit = [&](int k) -> int {
+        if (k * ncta >= units) return -1;
+        const int u = snake_unit(k, cta, ncta);
+        return u < units ? u : -1;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&ctl->q_full), 1);
@@ -331,6 +383,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(smem_u32(&ctl->o_empty[s]), kFwdRows);
         }
         mbar_init(smem_u32(&ctl->drain), 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(smem_u32(&ctl->unit_full[i]), 1);
+            mbar_init(smem_u32(&ctl->unit_empty[i]), kUnitReaders);
+        }
         ctl->abort = 0;
         fence_mbar_init();
     }
@@ -364,9 +420,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             uint32_t q_loads = 0;
             const uint32_t qbar = smem_u32(&ctl->q_full);
             bool ok = true;
-            for (int k = 0; k * ncta < units && ok; ++k) {
-                const int u = snake_unit(k, cta, ncta);
-                if (u >= units) continue;
+            for (int k = 0; ok; ++k) {
+                const int u = dyn ? fwd_publish_unit(ctl, vp.fetch, units, k, abort_flag, p.err, p.timeout_ns)
+                                  : static_unit(k);
+                if (u == -2) ok = false;
+                if (u < 0) break;
                 int g;
                 SeqGeo geo;
                 SubTile st[2];
@@ -487,9 +545,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                               (accumulate || kk > 0) ? 1u : 0u);
             };
 
-            for (int k = 0; k * ncta < units && ok; ++k) {
-                const int u = snake_unit(k, cta, ncta);
-                if (u >= units) continue;
+            for (int k = 0; ok; ++k) {
+                const int u = dyn ? fwd_read_unit(ctl, k, true, abort_flag, p.err, p.timeout_ns) : static_unit(k);
+                if (u == -2) ok = false;
+                if (u < 0) break;
                 int g;
                 SeqGeo geo;
                 SubTile st[2];
@@ -568,9 +627,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             uint32_t land_uses[kStages];
             for (int i = 0; i < kStages; ++i) land_uses[i] = 0;
             bool ok = true;
-            for (int k = 0; k * ncta < units && ok; ++k) {
-                const int u = snake_unit(k, cta, ncta);
-                if (u >= units) continue;
+            for (int k = 0; ok; ++k) {
+                const int u = dyn ? fwd_read_unit(ctl, k, false, abort_flag, p.err, p.timeout_ns) : static_unit(k);
+                if (u == -2) ok = false;
+                if (u < 0) break;
                 int g;
                 SeqGeo geo;
                 SubTile st[2];
@@ -619,9 +679,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float sl2 = p.scale_log2;
         uint32_t sph = 0, oph = 0;
         bool ok = true;
-        for (int k = 0; k * ncta < units && ok; ++k) {
-            const int u = snake_unit(k, cta, ncta);
-            if (u >= units) continue;
+        for (int k = 0; ok; ++k) {
+            const int u = dyn ? fwd_read_unit(ctl, k, false, abort_flag, p.err, p.timeout_ns) : static_unit(k);
+            if (u == -2) ok = false;
+            if (u < 0) break;
             int g;
             SeqGeo geo;
             SubTile st[2];
@@ -892,7 +953,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 // kDevErrBadSeqlens and an empty list: nothing is computed, nothing is written.
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 4 * kPlanThreads;
-constexpr int kPlanHeaderInts = 64;  // 256 bytes
+constexpr int kPlanHeaderInts = 64;  // 256 bytes: ws[0] = unit count, ws[1] = fetch counter
+// Launches of up to this many sequences list their units sequence-major (longest sequence
+// first, each sequence's longest row levels first) for dynamic fetching: the units a CTA
+// takes next then belong to the few sequences in flight, whose K/V stays in L2.
+constexpr int kPlanMaxDynamicSeqs = kPlanThreads;
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
     gqa_fwd_varlen_plan_kernel(const FwdParams p, const FwdVarlenParams vp, int S, int max_q,
@@ -918,7 +983,67 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     if (bad) {
         if (tid == 0) {
             ws[0] = 0;
+            ws[1] = 0;
             atomicOr(p.err, kDevErrBadSeqlens);
+        }
+        return;
+    }
+    if (vp.dynamic) {
+        // sequence-major list: rank the sequences by key count (longest first, ties by index),
+        // give each its units' range by a scan over ranks, then write its units with the
+        // longest row levels first. One thread per sequence (S <= kPlanMaxDynamicSeqs).
+        int* key = hist;                     // [S] key counts
+        int* cnt_by_rank = hist + kPlanThreads;
+        const bool pair = (p.unit_flags & kUnitPairHeads) != 0;
+        const int rows_per_lvl = pair ? kFwdRows : 2 * kFwdRows;
+        int lq = 0, lk = 0, cnt = 0, rank = 0;
+        if (tid < S) {
+            int bq, rq, bk, rk;
+            fwd_seq_side(vp.cu_q, vp.len_q, vp.rows_q, tid, bq, rq, lq);
+            fwd_seq_side(vp.cu_k, vp.len_k, vp.rows_k, tid, bk, rk, lk);
+            cnt = (lq + rows_per_lvl - 1) / rows_per_lvl * vp.n_h;
+            key[tid] = lk;
+        }
+        __syncthreads();
+        if (tid < S) {
+            for (int o = 0; o < S; ++o) rank += key[o] > lk || (key[o] == lk && o < tid);
+            cnt_by_rank[rank] = cnt;
+        }
+        __syncthreads();
+        // exclusive scan of the counts over ranks: rank r starts after ranks 0 .. r-1
+        int v = tid < S ? cnt_by_rank[tid] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_sum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int x = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            warp_sum[lane] = x;
+        }
+        __syncthreads();
+        incl += warp > 0 ? warp_sum[warp - 1] : 0;
+        const int total = warp_sum[31];
+        __syncthreads();
+        cnt_by_rank[tid] = incl - v;  // exclusive offset of rank tid
+        __syncthreads();
+        if (tid < S && cnt > 0) {
+            int* list = ws + kPlanHeaderInts + cnt_by_rank[rank];
+            const int n_lvl_s = cnt / vp.n_h;
+            for (int lvl = n_lvl_s - 1; lvl >= 0; --lvl)
+                for (int h = 0; h < vp.n_h; ++h) *list++ = (tid * vp.n_lvl + lvl) * vp.n_h + h;
+        }
+        if (tid == 0) {
+            ws[0] = total;
+            ws[1] = 0;
         }
         return;
     }
@@ -975,7 +1100,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
         const int w = fwd_unit_work(st);
         if (w > 0) list[atomicAdd(&hist[min(w, kPlanBuckets - 1)], 1)] = (int)c;
     }
-    if (tid == 0) ws[0] = total;
+    if (tid == 0) {
+        ws[0] = total;
+        ws[1] = 0;
+    }
 }
 
 }  // namespace gqa

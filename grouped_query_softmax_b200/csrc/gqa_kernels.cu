@@ -124,6 +124,8 @@ static cudaError_t launch_fwd_varlen_d(const FwdVarlenLaunch& a, cudaStream_t st
     vp.rows_k = a.rows_k;
     vp.unit_count = a.ws;
     vp.unit_list = a.ws + kPlanHeaderInts;
+    vp.fetch = a.ws + 1;
+    vp.dynamic = a.S <= kPlanMaxDynamicSeqs;
     vp.o_sb = a.o_sb;
     vp.o_sh = a.o_sh;
     vp.o_st = a.o_st;

@@ -321,3 +321,29 @@ def test_chunked_prefill_over_a_paged_cache(gqa, case):
     _sync_ok(gqa)
     ref = ov.attention_varlen(_head_major(q), k, v, S, cu_q=cu_q, len_k=lk, window=w)
     _check_packed(from_dev(o), ref, cu_q, f"paged prefill {case}")
+
+
+@pytest.mark.parametrize("S, q_hi, k_extra_hi", [
+    (40, 700, 1500),    # few sequences: units listed sequence-major and fetched dynamically
+    (1100, 4, 6),       # more sequences than the dynamic plan takes: the static longest-first order
+])
+def test_every_unit_computed_once(gqa, S, q_hi, k_extra_hi):
+    """The output starts as NaN: every row of every sequence must be written, by the unit that
+    owns it, and a second launch must give the same bits (the CTA that takes a unit varies in a
+    dynamically fetched launch, its result must not)."""
+    torch = torch_mod()
+    lq = gi.uniform_ints(5, gi.STREAM_LEN, S, 1, q_hi)
+    lk = lq + gi.uniform_ints(5, gi.STREAM_PREFIX, S, 0, k_extra_hi)
+    Hq, Hkv, D = 8, 2, 128
+    q, k, v, cu_q, cu_k = _packed(lq, lk, Hq, Hkv, D, seed=77)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    outs = []
+    for _ in range(2):
+        out = torch.full_like(qd, float("nan"))
+        gqa.attn_fwd_varlen(qd, kd, vd, cu_seqlens_q=_i32(cu_q), cu_seqlens_k=_i32(cu_k), out=out)
+        _sync_ok(gqa)
+        outs.append(bits_of(out))
+    assert np.array_equal(outs[0], outs[1])
+    got = gi.bf16_bits_to_f32(outs[0]).reshape(q.shape)
+    ref = ov.attention_varlen(_head_major(q), _head_major(k), _head_major(v), S, cu_q=cu_q, cu_k=cu_k)
+    _check_packed(got, ref, cu_q, f"{S} sequences")
