@@ -333,21 +333,27 @@ def long_pass(fn, res, long_s, world, dev):
 
 
 def measure_prefill(w, steps, warmup, world, dev, e2e_steps=0, inputs=None, long_s=0.0):
-    """gqa_attn_fwd over `steps` calls on inputs resident in HBM; optionally a long pass of
-    the same call, and the host-memory call end to end (e2e_steps > 0)."""
+    """attn_fwd (gqa_attn_fwd_split, which splits the last wave's key tiles over the SMs when
+    its plan says so, and is gqa_attn_fwd otherwise) over `steps` calls on inputs resident in
+    HBM, its workspace allocated once; optionally a long pass of the same call, and the
+    host-memory call end to end (e2e_steps > 0)."""
     import torch
     import grouped_query_softmax_b200 as gqa
     q, k, v = inputs if inputs is not None else w.make()
     qd, kd, vd = to_device(q, dev), to_device(k, dev), to_device(v, dev)
     od = torch.empty_like(qd)
-    fn = lambda: gqa.attn_fwd(qd, kd, vd, out=od, window=w.window)
+    need = gqa.gqa_attn_fwd_split_workspace_bytes(w.B, w.Hq, w.Hkv, w.Tq, w.Tk, w.D, w.window)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    fn = lambda: gqa.attn_fwd(qd, kd, vd, out=od, window=w.window, workspace=ws)
     ms, t0, t1 = timed(fn, steps, warmup, world, dev)
-    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": steps, "steps": steps}
+    # a split launch is the forward kernel and the merge of the pieces
+    res = {"ms_total": ms, "t0": t0, "t1": t1, "launches": steps * (2 if need else 1), "steps": steps,
+           "split_bytes": need}
     long_pass(fn, res, long_s, world, dev)
     st = gqa.gqa_get_device_error(torch.cuda.current_stream().cuda_stream)
     if st != gqa.GQA_OK:
         raise RuntimeError(f"device error after prefill timing: {gqa.gqa_status_string(st)}")
-    del qd, kd, vd, od
+    del qd, kd, vd, od, ws
     torch.cuda.empty_cache()
     if e2e_steps <= 0:
         return res

@@ -67,10 +67,11 @@ struct FwdParams {
     float* lse;  // nullable
     uint32_t* err;
     unsigned long long timeout_ns;
-    // split launches: units from split_whole on are parts, split_k per unit, each covering
-    // a k-th of that unit's key tiles; they write fp32 O / l rows to part and their
-    // log2-domain log-sum-exp to part_lse (split_k <= 1: no parts)
-    int split_whole, split_k;
+    // split launches (split_slices > 0): the first split_whole units run whole, the other
+    // units - split_whole are cut into key-tile pieces over split_slices slices (entries
+    // split_whole + 2 * slice + piece), in split_group lanes of units that share K/V; pieces
+    // write fp32 O / l rows to part and their log2-domain log-sum-exp to part_lse
+    int split_whole, split_slices, split_group;
     float* part;
     float* part_lse;
 };
@@ -126,6 +127,7 @@ struct FwdSmem {
         uint64_t unit_full[4];   // dynamic unit fetch: the producer publishes the CTA's k-th unit
         uint64_t unit_empty[4];  // in slot k % 4; its readers release the slot
         int unit_ring[4];
+        int split_entry[2];      // split launch: this CTA's pieces (fwd_split_entry), -1: none
         uint32_t tmem_base;
         uint32_t abort;
     };
@@ -199,23 +201,54 @@ __device__ __forceinline__ void fwd_decode_unit(const FwdParams& p, int u, int& 
     fwd_fill_subtile(st[1], p.Tq, off, p.window);
 }
 
-// Part index of unit u of a split launch (-1 for a whole unit) and the unit it is a part of.
-__device__ __forceinline__ int fwd_split_part(const FwdParams& p, int u, int& base) {
-    if (p.split_k <= 1 || u < p.split_whole) {
-        base = u;
-        return -1;
-    }
-    const int v = u - p.split_whole;
-    const int su = v / p.split_k;
-    base = p.split_whole + su;
-    return v - su * p.split_k;
+// a b / c for non-negative a, b and positive c, in 32-bit arithmetic when it fits.
+__device__ __forceinline__ long long fwd_muldiv(long long a, long long b, long long c) {
+    const long long x = a * b;
+    if (x <= 0x7fffffffLL && c <= 0x7fffffffLL) return (long long)((uint32_t)x / (uint32_t)c);
+    return x / c;
 }
 
-// Part `part` of `k` of a unit covers key tiles [n * part / k, n * (part + 1) / k) of its
-// n = longest sub-tile's tiles; each sub-tile keeps the tiles of its own range inside it.
-__device__ __forceinline__ void fwd_clamp_part(SubTile (&st)[2], int part, int k) {
-    const int n_max = max(st[0].n_kv, st[1].n_kv);
-    const int j0 = n_max * part / k, j1 = n_max * (part + 1) / k;
+// Split launches. The S = units - split_whole last units form S / L groups of L consecutive
+// units (the row levels of one KV head, which share its K/V; L = split_group); each group is
+// laid out as N ticks (N = key tiles of the launch's last row, a bound on every unit's tiles)
+// and the S / L groups end to end as T = (S / L) N ticks, dealt out as m = split_slices / L
+// equal runs. Slice i = j L + lane takes run j of the unit in lane `lane` of each group it
+// reaches, so the L CTAs of one run read the same keys of one head at the same time (L2
+// hits). S / L <= m: a run crosses at most one group boundary. Piece 0 of slice i lies in the
+// group holding the run's first tick, piece 1 (when the run crosses) in the next group. A
+// piece covering ticks [a, b) of a unit with n key tiles takes tiles [a n / N, b n / N), so
+// adjacent pieces tile every unit exactly.
+__device__ __forceinline__ bool fwd_split_piece(const FwdParams& p, int slot, int& su, int& a, int& b) {
+    const int L = p.split_group;
+    const int m = p.split_slices / L;
+    const long long N = (p.Tk - 1) / kFwdKeys + 1;
+    const long long T = (long long)((p.units - p.split_whole) / L) * N;
+    const int i = slot >> 1;
+    const int j = i / L, lane = i - j * L;
+    const long long lo = fwd_muldiv(T, j, m), hi = fwd_muldiv(T, j + 1, m);
+    const long long g0 = fwd_muldiv(lo, 1, N);
+    long long gr;
+    if (slot & 1) {
+        const long long start = (g0 + 1) * N;
+        if (hi <= start) return false;
+        gr = g0 + 1;
+        a = 0;
+        b = (int)(hi - start);
+    } else {
+        if (hi <= lo) return false;
+        gr = g0;
+        a = (int)(lo - g0 * N);
+        b = (int)(min(hi, (g0 + 1) * N) - g0 * N);
+    }
+    su = (int)(gr * L + lane);
+    return true;
+}
+
+// Keep key tiles [n a / N, n b / N) of a unit whose longest sub-tile has n tiles; each
+// sub-tile keeps the tiles of its own range inside them (none: n_kv = 0).
+__device__ __forceinline__ void fwd_clamp_ticks(SubTile (&st)[2], int a, int b, int N) {
+    const long long n_max = max(st[0].n_kv, st[1].n_kv);
+    const int j0 = (int)fwd_muldiv(n_max, a, N), j1 = (int)fwd_muldiv(n_max, b, N);
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
         if (st[s].n_kv == 0) continue;
@@ -223,6 +256,24 @@ __device__ __forceinline__ void fwd_clamp_part(SubTile (&st)[2], int part, int k
         st[s].n_kv = min(st[s].n_kv, j1);
         if (st[s].j_begin >= st[s].n_kv) st[s].n_kv = 0;
     }
+}
+
+// Unit u of a dense launch: a whole unit, or (u >= split_whole in a split launch) a piece;
+// an absent piece comes back with no tiles. Returns the split slot (-1: a whole unit).
+__device__ __forceinline__ int fwd_dense_unit(const FwdParams& p, int u, int& b, int& g, SubTile (&st)[2]) {
+    if (p.split_slices <= 0 || u < p.split_whole) {
+        fwd_decode_unit(p, u, b, g, st);
+        return -1;
+    }
+    const int slot = u - p.split_whole;
+    int su = 0, ta = 0, tb = 0;
+    const bool has = fwd_split_piece(p, slot, su, ta, tb);
+    fwd_decode_unit(p, p.split_whole + su, b, g, st);
+    if (has)
+        fwd_clamp_ticks(st, ta, tb, (p.Tk - 1) / kFwdKeys + 1);
+    else
+        st[0].n_kv = st[1].n_kv = 0;
+    return slot;
 }
 
 // One sequence side: batch index, first row and length.
@@ -279,10 +330,8 @@ __device__ __forceinline__ void fwd_unit(const FwdParams& p, const FwdVarlenPara
     if constexpr (kVarlen) {
         fwd_varlen_unit(p, vp, __ldg(vp.unit_list + u), geo, g, st);
     } else {
-        int b, base;
-        const int part = fwd_split_part(p, u, base);
-        fwd_decode_unit(p, base, b, g, st);
-        if (part >= 0) fwd_clamp_part(st, part, p.split_k);
+        int b;
+        fwd_dense_unit(p, u, b, g, st);
         geo.b_q = geo.b_k = b;
         geo.r_q = geo.r_k = 0;
         geo.len_q = p.Tq;
@@ -294,6 +343,23 @@ __device__ __forceinline__ void fwd_unit(const FwdParams& p, const FwdVarlenPara
 // unit list (i, 2n-1-i, 2n+i, ...), so each CTA's total work is nearly equal.
 __device__ __forceinline__ int snake_unit(int k, int i, int n) {
     return k * n + ((k & 1) ? (n - 1 - i) : i);
+}
+
+// The k-th entry of persistent CTA i of n in a split launch: its split_whole / n whole units
+// on the boustrophedon walk, then the pieces of slice i that hold key tiles (-1: none left).
+__device__ __forceinline__ int fwd_split_entry(const FwdParams& p, int k, int i, int n) {
+    const int full = p.split_whole / n;
+    if (k < full) return snake_unit(k, i, n);
+    if (i >= p.split_slices) return -1;
+    int want = k - full;
+    for (int piece = 0; piece < 2; ++piece) {
+        const int u = p.split_whole + 2 * i + piece;
+        int b, g;
+        SubTile st[2];
+        fwd_dense_unit(p, u, b, g, st);
+        if (fwd_unit_work(st) > 0 && want-- == 0) return u;
+    }
+    return -1;
 }
 
 // The k-th unit of a persistent CTA as a list index, -1 when the CTA has no more, -2 when a
@@ -363,6 +429,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const bool dyn = kVarlen && vp.dynamic != 0;
     // static launches: the k-th unit of this CTA on the boustrophedon walk (-1: none left)
     auto static_unit = [&](int k) -> int {
+        if (!kVarlen && p.split_slices > 0) {
+            const int full = p.split_whole / ncta;
+            if (k < full) return snake_unit(k, cta, ncta);
+            return k - full < 2 ? ctl->split_entry[k - full] : -1;
+        }
         if (k * ncta >= units) return -1;
         const int u = snake_unit(k, cta, ncta);
         return u < units ? u : -1;
@@ -388,6 +459,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(smem_u32(&ctl->unit_empty[i]), kUnitReaders);
         }
         ctl->abort = 0;
+        if (!kVarlen && p.split_slices > 0) {
+            const int full = p.split_whole / ncta;
+            ctl->split_entry[0] = fwd_split_entry(p, full, cta, ncta);
+            ctl->split_entry[1] = fwd_split_entry(p, full + 1, cta, ncta);
+        }
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -677,6 +753,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t tS = tmem + lane_sel + (uint32_t)(s * 128);
         const uint32_t tO = tmem + lane_sel + 256u + (uint32_t)(s * D);
         const float sl2 = p.scale_log2;
+        if (!kVarlen && cta < p.split_slices) {
+            // this CTA's partial rows start as "no key": a piece (or sub-tile) that holds no
+            // tile leaves them so, and the merge kernel skips them (the epilogue below, in this
+            // same thread, overwrites the rows it computes)
+            for (int i = 0; i < 2; ++i) p.part_lse[((size_t)(2 * cta + i) * 2 + s) * kFwdRows + r] = -INFINITY;
+        }
         uint32_t sph = 0, oph = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -808,16 +890,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 break;
             oph ^= 1u;
             tc_fence_after_sync();
-            int part = -1, base_u = u;
-            if constexpr (!kVarlen) part = fwd_split_part(p, u, base_u);
-            if (part >= 0) {
-                // a part of a split unit: fp32 O / l and the log2-domain log-sum-exp of this
-                // row over the part's keys (a row that saw none writes zeros and -inf); the
-                // combine kernel merges the parts
-                const size_t prow = ((size_t)(u - p.split_whole) * 2 + s) * kFwdRows + r;
+            if (!kVarlen && p.split_slices > 0 && u >= p.split_whole) {
+                // a piece of a split unit: fp32 O / l and the log2-domain log-sum-exp of this
+                // row over the piece's keys (a row that saw none writes zeros and -inf); the
+                // combine kernel merges the pieces
+                // rows chunk-major (float4 chunk e of row r at e * 128 + r): a warp's store
+                // of one chunk of its 32 rows is one contiguous 512-byte run
+                const size_t pblk = (size_t)(u - p.split_whole) * 2 + s;
+                const size_t prow = pblk * kFwdRows + r;
                 const bool any = l > 0.f;
                 const float inv_l = any ? 1.f / l : 0.f;
-                float4* dst = reinterpret_cast<float4*>(p.part + prow * D);
+                float4* dst = reinterpret_cast<float4*>(p.part + pblk * kFwdRows * D) + r;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t orr[32];
@@ -826,7 +909,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     reg_fence32(orr);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        dst[c * 8 + e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
+                        dst[(c * 8 + e) * kFwdRows] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
                                                      __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
                 }
                 tc_fence_before_sync();
@@ -881,67 +964,94 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 
 // ---------------------------------------------------------------- split-launch merge
-// Row r of sub-tile s of split unit su has split_k partial rows: fp32 O / l over a k-th of
-// its keys and the log2-domain log-sum-exp of those keys. With M the largest of them and
-// w_q = 2^(lse_q - M), the row is O = sum_q w_q O_q / sum_q w_q with log-sum-exp
-// M + log2(sum_q w_q): the same merge as the split-KV decode partials, in fixed part order.
-// One warp per row; each lane merges D / 32 consecutive columns.
+// Row r of sub-tile s of split unit su has one partial row per slice that reaches the unit:
+// fp32 O / l over the piece's keys (stored chunk-major: float4 chunk e of row r of a (slot,
+// sub-tile) block at e * 128 + r) and the log2-domain log-sum-exp of those keys (-inf when the
+// piece held none of this row's keys, or no tile of the sub-tile, or is absent: the forward
+// kernel writes -inf first). With M the largest and w_q = 2^(lse_q - M), the row is
+// O = sum_q w_q O_q / sum_q w_q with log-sum-exp M + log2(sum_q w_q): the merge of the
+// split-KV decode partials, summed in slice order, so the result is fixed.
+// One warp per 32 rows x 32 columns of one (unit, sub-tile), a lane per row: lane t first
+// finds the slot of candidate run c0 + t, then every load of a chunk for the warp's rows is one
+// 512-byte run.
 constexpr int kCombineWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32)
-    gqa_fwd_split_combine_kernel(const FwdParams p, long long n_rows) {
+    gqa_fwd_split_combine_kernel(const FwdParams p, long long n_warps) {
     const long long w = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
-    if (w >= n_rows) return;  // n_rows = split units x 2 sub-tiles x 128 rows
+    if (w >= n_warps) return;  // n_warps = split units x 2 sub-tiles x 4 row quarters x D / 32
+    constexpr int kColGroups = D / 32;
     const int lane = threadIdx.x & 31;
-    const int su = (int)(w >> 8);
-    const int s = (int)(w >> 7) & 1;
-    const int r = (int)w & (kFwdRows - 1);
+    const int cc = (int)(w % kColGroups);
+    const long long wr = w / kColGroups;
+    const int su = (int)(wr >> 3);
+    const int s = (int)(wr >> 2) & 1;
+    const int r = (int)(wr & 3) * 32 + lane;
     int b, g;
     SubTile st[2];
     fwd_decode_unit(p, p.split_whole + su, b, g, st);
-    const int row = st[s].row0 + r;
-    if (st[s].n_kv == 0 || row >= p.Tq) return;  // no such sub-tile, or a row past T_q
-    const int k = p.split_k;
-    const size_t base = ((size_t)su * k * 2 + s) * kFwdRows + r;  // part q: base + q * 2 * 128
-    const size_t stride = 2 * kFwdRows;
+    const SubTile me = s ? st[1] : st[0];
+    if (me.n_kv == 0 || me.row0 + (r & ~31) >= p.Tq) return;  // no such sub-tile, or rows past T_q
+    // runs c0 .. c1-1 of this unit's lane reach its group's ticks [x0, x1): c0 is the last
+    // one starting at or before x0, c1 the first one starting at or after x1
+    const int L = p.split_group;
+    const int m = p.split_slices / L;
+    const int gr = su / L, ln = su - gr * L;
+    const long long N = (p.Tk - 1) / kFwdKeys + 1;
+    const long long T = (long long)((p.units - p.split_whole) / L) * N;
+    const long long x0 = gr * N, x1 = x0 + N;
+    const int c0 = (int)fwd_muldiv((x0 + 1) * m - 1, 1, T);
+    const int c1 = (int)min((long long)m, fwd_muldiv(x1 * m + T - 1, 1, T));
+    auto slot_of = [&](int c) { return 2 * (c * L + ln) + (fwd_muldiv(T, c, m) < x0 ? 1 : 0); };
     float M = -INFINITY;
-    for (int q = 0; q < k; ++q) M = fmaxf(M, p.part_lse[base + q * stride]);
-    constexpr int kPer = D / 32;
-    float acc[kPer];
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-    float wsum = 0.f;
-    for (int q = 0; q < k; ++q) {
-        const float lq = p.part_lse[base + q * stride];
-        if (lq == -INFINITY) continue;  // the part held no key of this row
-        const float wq = ex2_approx(lq - M);
-        wsum += wq;
-        const float* src = p.part + (base + q * stride) * D + lane * kPer;
-        if constexpr (kPer == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            acc[0] += wq * v.x;
-            acc[1] += wq * v.y;
-            acc[2] += wq * v.z;
-            acc[3] += wq * v.w;
-        } else {
-            const float2 v = *reinterpret_cast<const float2*>(src);
-            acc[0] += wq * v.x;
-            acc[1] += wq * v.y;
+    for (int cb = c0; cb < c1; cb += 32) {
+        const int mine = cb + lane < c1 ? slot_of(cb + lane) : 0;
+        const int n = min(32, c1 - cb);
+        for (int t = 0; t < n; ++t) {
+            const size_t blk = (size_t)__shfl_sync(0xffffffffu, mine, t) * 2 + s;
+            M = fmaxf(M, p.part_lse[blk * kFwdRows + r]);
         }
     }
-    const float inv = 1.f / wsum;  // > 0: every row sees at least one key in some part
-    __nv_bfloat16* out = p.o + (((size_t)b * p.Hq + st[s].head) * (size_t)p.Tq + row) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-        uint2 pk;
-        pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-        pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-        *reinterpret_cast<uint2*>(out) = pk;
-    } else {
-        *reinterpret_cast<uint32_t*>(out) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    const int row = me.row0 + r;
+    float wsum = 0.f;
+    __nv_bfloat16* out = p.o + (((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row) * D;
+    {
+        float acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        for (int cb = c0; cb < c1; cb += 32) {
+            const int mine = cb + lane < c1 ? slot_of(cb + lane) : 0;
+            const int n = min(32, c1 - cb);
+            for (int t = 0; t < n; ++t) {
+                const size_t blk = (size_t)__shfl_sync(0xffffffffu, mine, t) * 2 + s;
+                const float lq = p.part_lse[blk * kFwdRows + r];
+                const float wq = lq == -INFINITY ? 0.f : ex2_approx(lq - M);
+                wsum += wq;
+                const float4* src = reinterpret_cast<const float4*>(p.part + blk * kFwdRows * D) + r;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 v = src[(cc * 8 + e) * kFwdRows];
+                    acc[4 * e] += wq * v.x;
+                    acc[4 * e + 1] += wq * v.y;
+                    acc[4 * e + 2] += wq * v.z;
+                    acc[4 * e + 3] += wq * v.w;
+                }
+            }
+        }
+        if (row < p.Tq) {
+            const float inv = 1.f / wsum;  // > 0: every row sees at least one key in some piece
+            uint4 v4[4];
+            uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+            uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = v4[e];
+        }
     }
-    if (p.lse != nullptr && lane == 0)
-        p.lse[((size_t)b * p.Hq + st[s].head) * (size_t)p.Tq + row] = (M + __log2f(wsum)) * 0.69314718055994530942f;
+    if (p.lse != nullptr && cc == 0 && row < p.Tq)
+        p.lse[((size_t)b * p.Hq + me.head) * (size_t)p.Tq + row] = (M + __log2f(wsum)) * 0.69314718055994530942f;
 }
 
 // ---------------------------------------------------------------- variable-length plan

@@ -190,7 +190,7 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
     gqa::FwdLaunch a{};
     a.window = window >= Tk ? 0 : window;  // a window covering every key is plain causal
-    a.split_k = 1;
+    a.split_slices = 0;
     if (allow_split) {
         int sms = 0;
         if ((st = current_sms(&sms)) != GQA_OK) return st;
@@ -199,7 +199,7 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float*
         if (need > 0) {
             if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
                 return GQA_ERR_WORKSPACE;
-            a.split_k = sp.k;
+            a.split_slices = sp.slices;
             a.part = static_cast<float*>(workspace);
         }
     }
@@ -548,11 +548,11 @@ gqa_status gqa_get_device_error(void* stream) {
 }
 
 gqa_status gqa_testing_fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window, int sms,
-                                      int* out_k, long long* out_whole, long long* out_split, long long* out_units) {
-    if (!out_k || !out_whole || !out_split || !out_units || sms < 1 || window < 0) return GQA_ERR_INVALID_ARGUMENT;
+                                      int* out_slices, long long* out_whole, long long* out_split, long long* out_units) {
+    if (!out_slices || !out_whole || !out_split || !out_units || sms < 1 || window < 0) return GQA_ERR_INVALID_ARGUMENT;
     if (check_common(B, Hq, Hkv, Tq, Tk, D) != GQA_OK) return GQA_ERR_INVALID_ARGUMENT;
     const gqa::FwdSplitPlan sp = gqa::fwd_split_plan(B, Hq, Hkv, Tq, Tk, window >= Tk ? 0 : window, sms);
-    *out_k = sp.k;
+    *out_slices = sp.slices;
     *out_whole = sp.whole;
     *out_split = sp.split;
     *out_units = gqa::fwd_units(B, Hq, Hkv, Tq);

@@ -2,6 +2,8 @@
 // unit (gqa_kernels.cu). Not installed, not part of the ABI.
 #pragma once
 
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -15,9 +17,10 @@ struct FwdLaunch {
     float scale;
     void* o;
     float* lse;
-    // split launch (fwd_split_plan): the last units' key tiles in split_k parts, whose
-    // fp32 partials go to `part` and are merged by a second kernel; split_k <= 1: none
-    int split_k;
+    // split launch (fwd_split_plan): the last units' key tiles dealt out over
+    // split_slices slices, whose fp32 partials go to `part` and are merged by a second
+    // kernel; split_slices = 0: none
+    int split_slices;
     float* part;
 };
 
@@ -31,23 +34,32 @@ inline long long fwd_units(int B, int Hq, int Hkv, int Tq) {
 
 // Split plan of a dense forward launch on `sms` persistent CTAs. Only plain causal suffix
 // launches whose cached prefix is at least as long as the suffix qualify: their units all
-// have about the same number of key tiles n, so a last wave of r = units mod sms units
-// leaves sms - r CTAs idle for a whole unit. Those r units are cut into k parts of about
-// n / k tiles (at least 2), which the persistent CTAs take after the whole units; k (at
-// most 8) minimises the estimated makespan (whole waves x n + part waves x (n / k + c),
-// c = kFwdSplitPartCost tiles standing for a part's fixed cost: its Q load, pipeline fill,
-// fp32 partial rows and share of the merge) and is used only if that estimate beats no
-// split by 10 %. Partial rows: split units x k x 2 sub-tiles x 128 rows.
+// have about n key tiles (n = the last row's), so a last wave of r = units mod sms units
+// would leave sms - r CTAs idle for most of a unit. The full waves run whole; the last r
+// units' key tiles are dealt out as `slices` equal runs of consecutive tiles, one per CTA,
+// cut at unit boundaries into pieces whose fp32 partial rows a second kernel merges. Units
+// come in groups of `group` (the row levels of one KV head, listed together); when the whole
+// units fill whole groups, each run covers the same keys of every unit of a group on
+// `group` CTAs at once, and slices is a multiple of group. Bounds: r <= slices <= min(sms,
+// r n / 2, 29 r): at least two tiles a run, at most 29 runs a unit. Estimated makespan in
+// key tiles: full x n + r n / slices + c per piece of the busiest slice (two unless slices
+// is a multiple of r, when no run crosses a unit boundary), c = kFwdSplitPartCost for a
+// piece's fixed cost (its Q load, pipeline fill, fp32 partial rows and share of the merge).
+// The best slice count is used when it beats the unsplit (full + 1) x n by the factor
+// kFwdSplitGain. Partial rows: slices x 2 pieces x 2 sub-tiles x 128 rows.
 struct FwdSplitPlan {
-    int k = 1;           // parts per split unit (1: no split)
+    int slices = 0;      // 0: no split
+    int group = 1;       // units per group of the slice lanes
     long long whole = 0; // units run whole (they come first in the unit list)
-    long long split = 0; // units cut into k parts
-    long long rows = 0;  // partial rows written to the workspace
+    long long split = 0; // units cut into pieces
+    long long rows = 0;  // partial rows in the workspace
 };
-constexpr int kFwdSplitMaxParts = 8;
-// Fixed cost of a part, in key tiles: the MHA suffix workload (256 units of 64 tiles on 148
-// SMs) measured 2.5 % slower split in 4 than whole, which puts it near 5 tiles.
 constexpr double kFwdSplitPartCost = 5.0;
+constexpr double kFwdSplitGain = 0.95;
+constexpr int kFwdSplitMaxPerUnit = 29;
+inline double fwd_split_cost(long long n, long long full, long long r, long long slices) {
+    return (double)full * n + (double)(r * n) / slices + kFwdSplitPartCost * (slices % r == 0 ? 1 : 2);
+}
 inline FwdSplitPlan fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int window, int sms) {
     FwdSplitPlan sp;
     const long long units = fwd_units(B, Hq, Hkv, Tq);
@@ -55,23 +67,29 @@ inline FwdSplitPlan fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int w
     if (window > 0 || Tk - Tq < Tq || sms <= 0 || units <= 0) return sp;
     const long long n = (Tk - 1) / 128 + 1;  // key tiles of a unit's last row
     const long long full = units / sms, r = units % sms;
-    if (r == 0) return sp;
+    if (r == 0 || n < 4) return sp;
+    // these launches list units head by head: the row levels of one head (pair) together
+    const int G = Hq / Hkv;
+    const int n_qt = (Tq + 127) / 128;
+    long long group = G % 2 == 0 ? n_qt : (n_qt + 1) / 2;
+    if ((full * sms) % group != 0) group = 1;
+    const long long top = std::min<long long>(std::min<long long>(sms, r * n / 2), r * kFwdSplitMaxPerUnit);
     const double base = (double)(full + 1) * n;
     double best = base;
-    int best_k = 1;
-    for (int k = 2; k <= kFwdSplitMaxParts && n / k >= 2; ++k) {
-        const long long part_waves = (r * k + sms - 1) / sms;
-        const double cost = (double)full * n + (double)part_waves * ((double)n / k + kFwdSplitPartCost);
+    long long best_s = 0;
+    for (long long s = (r + group - 1) / group * group; s <= top; s += group) {
+        const double cost = fwd_split_cost(n, full, r, s);
         if (cost < best) {
             best = cost;
-            best_k = k;
+            best_s = s;
         }
     }
-    if (best_k == 1 || best > 0.9 * base) return sp;
-    sp.k = best_k;
-    sp.whole = units - r;
+    if (best_s == 0 || best > kFwdSplitGain * base) return sp;
+    sp.slices = (int)best_s;
+    sp.group = (int)group;
+    sp.whole = full * sms;
     sp.split = r;
-    sp.rows = r * best_k * 2 * 128;
+    sp.rows = best_s * 2 * 2 * 128;
     return sp;
 }
 // Workspace of a split launch: fp32 partial O rows [rows, D], then their log2-domain
@@ -80,7 +98,7 @@ inline size_t fwd_split_lse_offset(long long rows, int D) {
     return ((size_t)rows * D * sizeof(float) + 255) & ~(size_t)255;
 }
 inline size_t fwd_split_workspace_bytes(const FwdSplitPlan& sp, int D) {
-    if (sp.k <= 1) return 0;
+    if (sp.slices <= 0) return 0;
     return fwd_split_lse_offset(sp.rows, D) + (size_t)sp.rows * sizeof(float);
 }
 

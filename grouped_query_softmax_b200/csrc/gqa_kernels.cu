@@ -59,16 +59,18 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     FwdSplitPlan sp;
-    p.split_k = 1;
-    if (a.split_k > 1) {
+    p.split_slices = 0;
+    p.split_whole = 0;
+    p.split_group = 1;
+    if (a.split_slices > 0) {
         // the caller sized its workspace with the same plan on the same device
         sp = fwd_split_plan(a.B, a.Hq, a.Hkv, a.Tq, a.Tk, a.window, sms);
-        if (sp.k != a.split_k || !a.part || units != sp.whole + sp.split) return cudaErrorInvalidValue;
+        if (sp.slices != a.split_slices || !a.part || units != sp.whole + sp.split) return cudaErrorInvalidValue;
         p.split_whole = (int)sp.whole;
-        p.split_k = sp.k;
+        p.split_slices = sp.slices;
+        p.split_group = sp.group;
         p.part = a.part;
         p.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(a.part) + fwd_split_lse_offset(sp.rows, D));
-        units = sp.whole + sp.split * sp.k;
     }
     if (units <= 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.units = (int)units;
@@ -81,16 +83,17 @@ static cudaError_t launch_fwd_d(const FwdLaunch& a, cudaStream_t stream) {
     e = cudaFuncGetAttributes(&fa, gqa_fwd_sm100_kernel<D, false>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
-    // persistent: one CTA per SM (shared memory and TMEM allow exactly one)
-    const unsigned grid = (unsigned)std::min<long long>(units, sms > 0 ? sms : 1);
+    // persistent: one CTA per SM (shared memory and TMEM allow exactly one); a split launch
+    // has one CTA per SM exactly, as its plan assumes
+    const unsigned grid = p.split_slices > 0 ? (unsigned)sms : (unsigned)std::min<long long>(units, sms > 0 ? sms : 1);
     gqa_fwd_sm100_kernel<D, false><<<grid, kFwdThreads, smem, stream>>>(a.tm_q, a.tm_k, a.tm_v, p,
                                                                          FwdVarlenParams{});
     e = cudaGetLastError();
-    if (e != cudaSuccess || p.split_k <= 1) return e;
-    // merge the parts of the split units (stream order makes their partials visible)
-    const long long rows = sp.split * 2 * kFwdRows;
-    const long long blocks = (rows + kCombineWarps - 1) / kCombineWarps;
-    gqa_fwd_split_combine_kernel<D><<<(unsigned)blocks, kCombineWarps * 32, 0, stream>>>(p, rows);
+    if (e != cudaSuccess || p.split_slices <= 0) return e;
+    // merge the pieces of the split units (stream order makes their partials visible)
+    const long long warps = sp.split * 2 * (kFwdRows / 32) * (D / 32);
+    const long long blocks = (warps + kCombineWarps - 1) / kCombineWarps;
+    gqa_fwd_split_combine_kernel<D><<<(unsigned)blocks, kCombineWarps * 32, 0, stream>>>(p, warps);
     return cudaGetLastError();
 }
 

@@ -104,10 +104,12 @@ GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, 
  * Which launches split: plain causal suffix calls (window = 0) whose cached prefix is at
  * least as long as the suffix (T_k - T_q >= T_q). Their work units (pairs of 128-row query
  * tiles) all need about the same number of key tiles, so when their count is not a multiple
- * of the number of SMs the last wave of the persistent kernel leaves SMs idle. The units of
- * that last wave are then cut into 2 to 8 parts along the keys; each part writes its rows'
- * fp32 partial output and log-sum-exp to the workspace, and a second kernel merges them by
- * log-sum-exp (the same merge as decode's split-KV partials). The tile splitting that
+ * of the number of SMs the last wave of the persistent kernel leaves SMs idle. The full waves
+ * then run whole, and the key tiles of the last wave's units, laid end to end, are dealt out
+ * in equal runs of consecutive tiles, one run per SM; a run is cut at unit boundaries into
+ * pieces, each piece writes its rows' fp32 partial output and log-sum-exp to the workspace,
+ * and a second kernel merges them by log-sum-exp (the same merge as decode's split-KV
+ * partials). The tile splitting that
  * "A Visual Guide to Attention", section "Sources and execution", describes for one row is
  * here spread over CTAs.
  *

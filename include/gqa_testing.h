@@ -57,12 +57,13 @@ GQA_API gqa_status gqa_testing_fwd_host_fail_at(int chunk);
 
 /*
  * The split plan of gqa_attn_fwd_split for a device with `sms` SMs, for host-side tests:
- * *out_k parts per split unit (1 = no split), *out_whole units run whole, *out_split units
- * cut into *out_k parts, *out_units = all units. Touches no GPU. Returns
+ * *out_slices runs of key tiles the last units are dealt out in (0 = no split), *out_whole
+ * units run whole, *out_split units cut into pieces, *out_units = all units. Touches no GPU.
+ * Returns
  * GQA_ERR_INVALID_ARGUMENT for sizes gqa_attn_fwd_ex rejects, sms < 1 or a null pointer.
  */
 GQA_API gqa_status gqa_testing_fwd_split_plan(int B, int Hq, int Hkv, int Tq, int Tk, int D, int window, int sms,
-                                              int* out_k, long long* out_whole, long long* out_split,
+                                              int* out_slices, long long* out_whole, long long* out_split,
                                               long long* out_units);
 
 #ifdef __cplusplus

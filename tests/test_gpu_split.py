@@ -1,5 +1,5 @@
-"""GPU parity of gqa_attn_fwd_split: suffix launches whose last wave of work units is cut along
-the keys into parts, merged by log-sum-exp. Checked against the fp64 oracle, against the unsplit
+"""GPU parity of gqa_attn_fwd_split: suffix launches whose last wave of work units is dealt out
+over the SMs in runs of key tiles, cut into pieces at unit boundaries and merged by log-sum-exp. Checked against the fp64 oracle, against the unsplit
 call, for determinism, and for the workspace rules, all through the C ABI."""
 import numpy as np
 import pytest
@@ -16,6 +16,9 @@ SHAPES = [
     (1, 8, 8, 1024, 2048, 128, 0),    # prefix = suffix: some rows see no key in the last part
     (1, 8, 2, 600, 2500, 64, 0),      # D = 64, offset not tile-aligned
     (1, 16, 4, 256, 4096, 128, 0),    # 16 units of 32 key tiles
+    (7, 32, 32, 128, 4096, 128, 0),   # a whole wave, then slices crossing unit boundaries;
+                                      # one-sub-tile units (T_q = 128)
+    (7, 16, 16, 384, 4096, 64, 2),    # the same with D = 64, and units whose second sub-tile is absent
 ]
 
 
