@@ -112,7 +112,11 @@ struct FwdSmem {
     static constexpr int kStages = D == 128 ? 4 : 8;   // ring slots, each one K or one V tile
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = 2 * kTileBytes;
-    static constexpr int kCtlOff = kRingOff + kStages * kTileBytes;
+    // output staging: each softmax warp's 32 rows x 64 columns of bf16 (128 bytes a row), so
+    // the epilogue's global stores go out as whole row segments
+    static constexpr int kStageWarpBytes = 32 * 128;
+    static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
+    static constexpr int kCtlOff = kStageOff + 8 * kStageWarpBytes;
     struct Ctl {
         uint64_t q_full;
         uint64_t q_empty;
@@ -132,6 +136,7 @@ struct FwdSmem {
         uint32_t abort;
     };
     static constexpr int kBytes = kCtlOff + (int)sizeof(Ctl) + 1024;  // + alignment slack
+    static_assert(kBytes <= 232448, "shared memory above the 227 KB a CTA may have");
 };
 
 struct SubTile {
@@ -415,6 +420,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t sbase = raw_addr + pad;
     const uint32_t sQ = sbase + L::kQOff;
     const uint32_t sRing = sbase + L::kRingOff;
+    const uint32_t sStage = sbase + L::kStageOff;
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtlOff);
     volatile uint32_t* abort_flag = &ctl->abort;
 
@@ -920,32 +926,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int row = me.row0 + r;
             const bool row_ok = row < geo.len_q;
             const float inv_l = 1.f / l;
-            __nv_bfloat16* out;
-            if constexpr (kVarlen)
-                out = p.o + geo.b_q * vp.o_sb + me.head * vp.o_sh + (long long)(geo.r_q + row) * vp.o_st;
-            else
-                out = p.o + (((size_t)geo.b_q * p.Hq + me.head) * (size_t)p.Tq + (size_t)row) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                tmem_ld32(tO + c * 32, orr);
-                tc_wait_ld();
-                reg_fence32(orr);
-                uint4 v4[4];
-                uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pw[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
-                                        __uint_as_float(orr[2 * e + 1]) * inv_l);
-                if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = v4[e];
-                }
+            // row 0 of this warp's 32 output rows, and the row stride (elements)
+            __nv_bfloat16* out0;
+            long long ost;
+            if constexpr (kVarlen) {
+                out0 = p.o + geo.b_q * vp.o_sb + me.head * vp.o_sh + (long long)(geo.r_q + me.row0 + quad * 32) * vp.o_st;
+                ost = vp.o_st;
+            } else {
+                out0 = p.o + (((size_t)geo.b_q * p.Hq + me.head) * (size_t)p.Tq + (size_t)(me.row0 + quad * 32)) * D;
+                ost = D;
             }
-            // O_s has been read: the next unit's first P V may overwrite it
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&ctl->o_empty[s]));
+            const int rows_left = geo.len_q - me.row0 - quad * 32;  // of the warp's rows, those that exist
+            const uint32_t stg = sStage + (uint32_t)(warp - 4) * L::kStageWarpBytes;
+            // 64 columns at a time: O / l as bf16 into the warp's staging rows (16-byte chunk q of
+            // row t at chunk q ^ (t & 7), so 8 consecutive rows fill all banks), then back out as
+            // whole 128-byte row segments, 4 rows per store instruction
+#pragma unroll 1
+            for (int h = 0; h < D / 64; ++h) {
+                uint32_t pw[32];
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + h * 64 + c2 * 32, orr);
+                    tc_wait_ld();
+                    reg_fence32(orr);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pw[c2 * 16 + e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
+                                                      __uint_as_float(orr[2 * e + 1]) * inv_l);
+                }
+                if (h == D / 64 - 1) {
+                    // O_s has been read: the next unit's first P V may overwrite it
+                    tc_fence_before_sync();
+                    mbar_arrive(smem_u32(&ctl->o_empty[s]));
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    st_shared_v4(stg + lane * 128 + ((q ^ (lane & 7)) << 4), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2],
+                                 pw[4 * q + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int t = i * 4 + (lane >> 3), q = lane & 7;
+                    const uint4 v = ld_shared_v4(stg + t * 128 + ((q ^ (t & 7)) << 4));
+                    if (t < rows_left) *reinterpret_cast<uint4*>(out0 + (long long)t * ost + h * 64 + q * 8) = v;
+                }
+                __syncwarp();
+            }
             if (p.lse != nullptr && row_ok) {
                 const size_t li = kVarlen ? ((size_t)geo.b_q * p.Hq + me.head) * (size_t)vp.rows_q + geo.r_q + row
                                           : ((size_t)geo.b_q * p.Hq + me.head) * (size_t)p.Tq + row;
