@@ -944,16 +944,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll 1
             for (int h = 0; h < D / 64; ++h) {
                 uint32_t pw[32];
-#pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t orr[32];
-                    tmem_ld32(tO + h * 64 + c2 * 32, orr);
+                {
+                    uint32_t orr[2][32];
+                    tmem_ld32(tO + h * 64, orr[0]);
+                    tmem_ld32(tO + h * 64 + 32, orr[1]);
                     tc_wait_ld();
-                    reg_fence32(orr);
+                    reg_fence32(orr[0]);
+                    reg_fence32(orr[1]);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pw[c2 * 16 + e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
-                                                      __uint_as_float(orr[2 * e + 1]) * inv_l);
+                    for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pw[c2 * 16 + e] = pack_bf16x2(__uint_as_float(orr[c2][2 * e]) * inv_l,
+                                                          __uint_as_float(orr[c2][2 * e + 1]) * inv_l);
                 }
                 if (h == D / 64 - 1) {
                     // O_s has been read: the next unit's first P V may overwrite it
