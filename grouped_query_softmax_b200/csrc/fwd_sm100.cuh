@@ -148,6 +148,15 @@ struct SubTile {
     int lo_masked_end;  // KV tiles below this cross the lower edge of the window
 };
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // Key-tile bounds of one sub-tile whose rows sit at positions off + row0 ...
 __device__ __forceinline__ void fwd_fill_subtile(SubTile& st, int len_q, int off, int window) {
     st.j_begin = 0;
