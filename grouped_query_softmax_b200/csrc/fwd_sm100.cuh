@@ -849,25 +849,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const bool refresh = m_new > m + kRescaleThreshold;
                 // warp-uniform branch, rarely taken after a unit's first tile: the MUFU op for
                 // alpha stays off the common path (it would queue behind the exponentials)
+                float alpha = 1.f;  // < 2^-8 where this row's max moved, else exactly 1
                 if (__any_sync(0xffffffffu, refresh)) {
-                    const float alpha = refresh ? ex2_approx(m - m_new) : 1.f;
+                    alpha = refresh ? ex2_approx(m - m_new) : 1.f;
                     l *= alpha;
                     m = refresh ? m_new : m;
-                    if (j > me.j_begin) {
-                        // O_s has absorbed all earlier P V products (their completion is
-                        // ordered before S_j's commit); rescale this row in place.
-#pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t orr[32];
-                            tmem_ld32(tO + c * 32, orr);
-                            tc_wait_ld();
-                            reg_fence32(orr);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                            tmem_st32(tO + c * 32, orr);
-                        }
-                    }
                 }
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -895,6 +881,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     float a0, a1;
                     f2_unpack(s01, a0, a1);
                     l += a0 + a1;
+                }
+                if (__any_sync(0xffffffffu, alpha != 1.f) && j > me.j_begin) {
+                    // O_s has absorbed all earlier P V products (their completion is ordered
+                    // before S_j's commit) and this tile's P V waits for p_full below: rescale
+                    // this row in place, after the exponentials, when S no longer holds
+                    // registers, so all column chunks load behind one wait
+                    uint32_t orr[D / 32][32];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, orr[c]);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        reg_fence32(orr[c]);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[c][e] = __float_as_uint(__uint_as_float(orr[c][e]) * alpha);
+                        tmem_st32(tO + c * 32, orr[c]);
+                    }
                 }
                 tc_wait_st();
                 tc_fence_before_sync();
