@@ -23,7 +23,9 @@
 //                   rounded to bf16 and written over the first half of S in TMEM.
 //                   The running max is refreshed only when it grows by more than
 //                   2^8 (in the log2 domain), so O is rescaled rarely; the final
-//                   O / l and the log-sum-exp are exact whatever max was kept.
+//                   O / l and the log-sum-exp are exact whatever max was kept. The
+//                   epilogue stages each warp's bf16 rows in shared memory and
+//                   stores them as whole row segments.
 // Causal tile skipping: a sub-tile visits KV tiles 0 .. floor((off + last_row)/128)
 // only, and applies the mask only on tiles that cross its diagonal.
 #pragma once
