@@ -826,15 +826,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 reg_fence32(sr[2]);
                 reg_fence32(sr[3]);
                 if (diag) {
-                    // columns > lim are in the future; columns < lim_lo are before the window
-                    const int lim = pos - j * kFwdKeys;
-                    const int lim_lo = p.window > 0 ? lo - j * kFwdKeys : -1;
+                    if (j >= me.masked_from) {
+                        // the causal diagonal (sub-tile uniform): columns > lim are in the future
+                        const int lim = pos - j * kFwdKeys;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                        for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (c * 32 + e > lim || c * 32 + e < lim_lo) sr[c][e] = __float_as_uint(-INFINITY);
-                        }
+                            for (int e = 0; e < 32; ++e)
+                                if (c * 32 + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+                    }
+                    if (j < me.lo_masked_end) {
+                        // the window's lower edge (sub-tile uniform): columns < lim_lo are before it
+                        const int lim_lo = lo - j * kFwdKeys;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (c * 32 + e < lim_lo) sr[c][e] = __float_as_uint(-INFINITY);
+                    }
                 }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
