@@ -109,9 +109,8 @@ GQA_API gqa_status gqa_attn_fwd_ex(const void* q, const void* k, const void* v, 
  * in equal runs of consecutive tiles, one run per SM; a run is cut at unit boundaries into
  * pieces, each piece writes its rows' fp32 partial output and log-sum-exp to the workspace,
  * and a second kernel merges them by log-sum-exp (the same merge as decode's split-KV
- * partials). The tile splitting that
- * "A Visual Guide to Attention", section "Sources and execution", describes for one row is
- * here spread over CTAs.
+ * partials). The tile splitting that "A Visual Guide to Attention", section "Sources and
+ * execution", describes for one row is here spread over CTAs.
  *
  *   workspace, workspace_bytes  device memory of at least
  *            gqa_attn_fwd_split_workspace_bytes(B, Hq, Hkv, Tq, Tk, D, window) bytes (same
